@@ -1,0 +1,402 @@
+"""Benchmark of the MXFP4 MoE block-verify step on B200.
+
+One step = the whole hot path over one drafted batch: moe_route_topk ->
+moe_permute -> mxfp4_moe_ffn -> moe_combine -> block_accept_greedy (the
+batch-1 verify workload: 1 sequence x 8-token block, one MoE layer of
+hidden 7168, expert intermediate 2048, 256 experts, top-8; greedy acceptance
+over a 152064-token vocabulary).  Metric: verified tokens/s (= S*K / step
+time), with the HBM roofline of the expert FFN beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload batch1|serving|dflash16|multilayer|tiny]
+
+Multi-GPU: every rank verifies its own independent batch (the path has no
+exchange step); value = all ranks' tokens / the slowest rank's time.
+--impl reference times the CPU oracle (the reference arm of this repository)
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mxfp4_moe_block_b200 import synth  # noqa: E402
+
+METRIC = "verified tokens/s (MXFP4 MoE block-verify step)"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="batch1", choices=list(synth.SHAPES))
+    ap.add_argument("--variant", type=int, default=0, help="FFN kernel: 0 auto, 1 FMA, 2 tensor")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_tag():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mxfp4_moe_block_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload, variant_name):
+    """DRAM bytes per FFN call from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", f"ffn_{variant_name}_{workload}_traffic.txt")
+    try:
+        kv = {}
+        for line in open(p):
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("source_tag") != kernel_source_tag():
+            return None
+        return float(kv["dram_bytes_per_ffn_call"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        if shutil.which("nvidia-smi") is None:
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen(
+            ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+             "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+            stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload --
+
+class Workload:
+    """Seeded inputs of one verify step, resident in HBM."""
+
+    def __init__(self, sh, device, rank):
+        import mxfp4_moe_block_b200 as mm
+        self.mm = mm
+        self.sh = sh
+        self.dev = device
+        # every rank verifies its own batch: different activations / logits
+        self.sh_r = synth.Shape(**{**sh.__dict__, "seed": sh.seed + 7919 * rank})
+        s = self.sh_r
+        self.x_bits = synth.x_bf16_bits(s)
+        self.logits_np = synth.router_logits(s)
+        self.block_np = synth.block_logits(s)
+        self.draft_np = synth.greedy_drafts(s, self.block_np)
+        self.x = torch.from_numpy(self.x_bits.view(np.int16)).to(device).view(torch.bfloat16)
+        self.logits = torch.from_numpy(self.logits_np).to(device)
+        self.block = torch.from_numpy(self.block_np).to(device)
+        self.draft = torch.from_numpy(self.draft_np).to(device)
+        self.w = synth.weights_torch(sh, 0, device)      # model weights: same on every rank
+        T, k, E, H, I = s.T, s.k, s.E, s.H, s.I
+        i32 = dict(dtype=torch.int32, device=device)
+        self.idx = torch.empty((T, k), **i32)
+        self.tw = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.off = torch.empty(E + 1, **i32)
+        self.sp = torch.empty(T * k, **i32)
+        self.pr = torch.empty(T * k, **i32)
+        self.y = torch.empty((T * k, H), dtype=torch.float32, device=device)
+        self.ws = mm.alloc_workspace(T, k, H, I, device)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        self.acc = torch.empty(s.S, **i32)
+        self.nxt = torch.empty(s.S, **i32)
+
+    def step(self, variant, ev=None):
+        mm, s = self.mm, self.sh_r
+        if ev is not None:
+            ev[0].record()
+        mm.moe_route_topk(self.logits, s.k, self.idx, self.tw)
+        mm.moe_permute(self.idx, s.E, self.off, self.sp, self.pr)
+        if ev is not None:
+            ev[1].record()
+        mm.mxfp4_moe_ffn(self.x, s.k, *self.w, self.off, self.sp, y=self.y, workspace=self.ws,
+                         variant=variant)
+        if ev is not None:
+            ev[2].record()
+        mm.moe_combine(self.y, self.pr, self.tw, out=self.out)
+        mm.block_accept_greedy(self.block, self.draft, self.acc, self.nxt)
+        if ev is not None:
+            ev[3].record()
+
+    def activated_bytes(self):
+        off = self.off.cpu().numpy()
+        n_act = int((np.diff(off) > 0).sum())
+        return n_act * self.sh.expert_bytes(), n_act
+
+    def ffn_flops(self):
+        return 2.0 * self.sh_r.P * 3 * self.sh.H * self.sh.I
+
+
+def e2e_time(wl, variant, steps, warmup):
+    """Same step through the public API with host buffers: pinned inputs are
+    copied in and the results copied out inside the timed region."""
+    hx = torch.from_numpy(wl.x_bits.view(np.int16)).pin_memory()
+    hl = torch.from_numpy(wl.logits_np).pin_memory()
+    hb = torch.from_numpy(wl.block_np).pin_memory()
+    hd = torch.from_numpy(wl.draft_np).pin_memory()
+    ho = torch.empty(wl.out.shape, dtype=torch.bfloat16).pin_memory()
+    ha = torch.empty(wl.acc.shape, dtype=torch.int32).pin_memory()
+    hn = torch.empty(wl.nxt.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hl, hb, hd))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, ha, hn))
+
+    def one():
+        wl.x.view(torch.int16).copy_(hx, non_blocking=True)
+        wl.logits.copy_(hl, non_blocking=True)
+        wl.block.copy_(hb, non_blocking=True)
+        wl.draft.copy_(hd, non_blocking=True)
+        wl.step(variant)
+        ho.copy_(wl.out, non_blocking=True)
+        ha.copy_(wl.acc, non_blocking=True)
+        hn.copy_(wl.nxt, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+def oracle_step_seconds(sh, n_expert_sample=4, seed_shift=0):
+    """Time the CPU oracle on one step of the workload, with the expert FFN
+    on a sample of the active experts, scaled to all of them."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import accept as oacc
+    from oracle import moe as omoe
+    s = synth.Shape(**{**sh.__dict__, "seed": sh.seed + seed_shift})
+    x64 = synth.bf16_bits_to_f32(synth.x_bf16_bits(s)).astype(np.float64)
+    logits = synth.router_logits(s)
+    block = synth.block_logits(s)
+    draft = synth.greedy_drafts(s, block)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        idx, w, _ = omoe.route_topk(logits, s.k)
+        off, sp, pr = omoe.permute(idx, s.E)
+        t_route = time.perf_counter() - t0
+        act = [e for e in range(s.E) if off[e + 1] > off[e]]
+        sample = act[:: max(1, len(act) // n_expert_sample)][:n_expert_sample]
+        y = np.zeros((s.P, s.H))
+        t_ffn = 0.0
+        for e in sample:
+            r0, r1 = off[e], off[e + 1]
+            wts = (synth.weight_codes_np(s, "w13", e), synth.weight_scales_np(s, "w13", e),
+                   synth.weight_codes_np(s, "w2", e), synth.weight_scales_np(s, "w2", e))
+            t0 = time.perf_counter()            # weights are inputs: drawn before timing
+            _, y[r0:r1] = omoe.expert_ffn(x64[sp[r0:r1] // s.k], *wts, s.I)
+            t_ffn += time.perf_counter() - t0
+        t_ffn *= len(act) / len(sample)
+        t0 = time.perf_counter()
+        omoe.combine(y, pr, w)
+        oacc.greedy(block, draft)
+        t_rest = time.perf_counter() - t0
+    total = t_route + t_ffn + t_rest
+    return total, {"experts_active": len(act), "experts_sampled": len(sample)}
+
+
+# --------------------------------------------------------------------- main --
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    sh = synth.SHAPES[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        times = []
+        info = {}
+        for i in range(args.warmup + args.steps):
+            t, info = oracle_step_seconds(sh, seed_shift=0)
+            if i >= args.warmup:
+                times.append(t)
+        ms = 1e3 * statistics.mean(times)
+        value = sh.T / (ms / 1e3)
+        line = {
+            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": f"{sh.name}: H={sh.H} I={sh.I} E={sh.E} top-{sh.k}, "
+                                   f"S={sh.S} x K={sh.K}, V={sh.V}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"route+permute+combine+greedy in full; expert FFN on "
+                                       f"{info['experts_sampled']} of {info['experts_active']} "
+                                       f"active experts, time scaled to all"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import mxfp4_moe_block_b200 as mm
+    mm.lib()
+    wl = Workload(sh, dev, rank)
+    variant = args.variant
+
+    for _ in range(max(3, args.warmup)):
+        wl.step(variant)
+    torch.cuda.synchronize()
+    act_bytes, n_act = wl.activated_bytes()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        wl.step(variant, evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    ffn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    tail_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    e2e_ms, h2d, d2h = e2e_time(wl, variant, args.steps, 3)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peak, peak_kind = load_peaks()
+    achieved = act_bytes / (ffn_ms * 1e-3) / 1e9
+    vname = {0: "auto", 1: "fma", 2: "tensor"}[variant]
+    traffic = load_traffic(sh.name, vname)
+    tokens = sh.T * world
+    launches_per_step = 6 * (sh.layers if sh.layers > 1 else 1)
+    line = {
+        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4 weights, bf16 activations, f32 accumulate",
+        "data": "synthetic (seeded counter-based generator; random MXFP4 weights)",
+        "config": {"workload": f"{sh.name}: one MoE layer H={sh.H} I={sh.I} E={sh.E} top-{sh.k} SwiGLU, "
+                               f"S={sh.S} x K={sh.K} block, greedy over V={sh.V}",
+                   "global_batch_tokens": tokens, "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "inputs larger than L2: %.2f GB of expert weights read per step" % (act_bytes / 1e9),
+                   "ffn_variant": vname},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "mxfp4_moe_ffn (GEMM-1+SwiGLU and GEMM-2 launches)",
+                     "algorithmic_bytes": act_bytes, "active_experts": n_act,
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "breakdown_ms": {"route+permute": route_ms, "ffn": ffn_ms, "combine+greedy": tail_ms},
+        "ffn_tflops": wl.ffn_flops() / (ffn_ms * 1e-3) / 1e12,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, info = oracle_step_seconds(sh)
+        line["cpu_baseline"] = {
+            "value": sh.T / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"one step; expert FFN on {info['experts_sampled']} of "
+                      f"{info['experts_active']} active experts, time scaled to all"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,224 @@
+/*
+ * mxfp4_moe.h -- C ABI of the MXFP4 MoE block-verify library (B200, sm_100a).
+ *
+ * One speculative-decoding verify step of a mixture-of-experts target model:
+ * a drafted block of K tokens per sequence (T = S*K tokens) is routed top-k,
+ * grouped by expert, pushed through each expert's SwiGLU FFN whose weights
+ * are OCP MXFP4, weight-combined, and the block is accepted greedily or by
+ * rejection sampling.  Sources (page title, section):
+ *   [P1] "mimo-v2-5-speculative-decoding-draft-scheduling"
+ *   [P2] "如何评价小米6月9日发布的MiMo-V2.5-Pro-UltraSpeed模式？"
+ *   [P3] "MiMo-v2.5-Pro-UltraSpeed - infra 架构解读"
+ *   [P4] "mimo-tilert-1000tps-trillion-parameter-inference"
+ *   [OCP] OCP Microscaling Formats (MX) v1.0 (named by [P3] and [P4]).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument is a DEVICE pointer owned by the caller; the
+ *    library never allocates, frees or keeps a pointer after the call returns.
+ *  - Work is enqueued on `stream` and runs asynchronously; no call
+ *    synchronises except moe_get_device_status.
+ *  - Tensors are dense, row-major (last index fastest), with the shapes given.
+ *  - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *  - Return value: MOE_OK, or an error code.  Argument errors are detected on
+ *    the host and returned before anything is launched.  Errors only the
+ *    device can see (an expert id outside [0,E), a row with no probability
+ *    mass, a bounded wait that ran out) set a sticky device status word read
+ *    by moe_get_device_status; the kernel then skips the offending element
+ *    and never faults.  Inputs with NaN or infinity are unsupported: results
+ *    are unspecified, but no fault occurs.
+ */
+#ifndef MXFP4_MOE_H
+#define MXFP4_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size, k > E, ...          */
+  MOE_ERR_UNSUPPORTED = 2, /* shape outside what the kernels implement    */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed         */
+  MOE_ERR_WORKSPACE = 4,   /* workspace smaller than the query returned    */
+  MOE_ERR_DEVICE = 5       /* device status word set (see below)           */
+};
+
+/* Device-side error details (second argument of moe_get_device_status). */
+enum {
+  MOE_DEV_OK = 0,
+  MOE_DEV_BAD_EXPERT = 1,  /* moe_permute saw an expert id outside [0,E)   */
+  MOE_DEV_NO_MASS = 2,     /* block_accept_rejection: target row all zero  */
+  MOE_DEV_BAD_TOKEN = 3,   /* a draft token outside [0,V)                   */
+  MOE_DEV_TIMEOUT = 4      /* a bounded device wait ran out                */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *moe_status_string(int status);
+
+/* Library version, e.g. 1 00 00 -> 10000. */
+int moe_version(void);
+
+/*
+ * moe_route_topk -- top-k expert routing of T tokens over E experts.
+ *   Each token activates a few experts ([P4] "万亿参数推理为什么特别难");
+ *   the router keeps high precision ([P4] "第一层：FP4 选择性量化").  Rule:
+ *   expert i of a token is selected iff fewer than k experts j have
+ *   logit_j > logit_i or (logit_j == logit_i and j < i); selected experts are
+ *   listed by that rank (descending logit, ties to the lowest index).
+ *   Weights are softmax over the k selected logits, evaluated in double
+ *   precision and rounded once to float.
+ *   logits   [T, E] float   (finite)
+ *   topk_idx [T, k] int32   out
+ *   topk_w   [T, k] float   out
+ *   Limits: 1 <= k <= min(E, 32), 1 <= E <= 1024, T >= 0.
+ */
+int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
+                   float *topk_w, moe_stream_t stream);
+
+/*
+ * moe_permute -- stable grouping of the T*k (token, slot) pairs by expert.
+ *   Pair id p = t*k + j.  expert_offsets[e] .. expert_offsets[e+1] is the
+ *   range of sorted rows of expert e; sorted_pair lists pair ids expert by
+ *   expert, ascending inside an expert; pair_row is its inverse
+ *   (pair_row[sorted_pair[r]] == r).
+ *   topk_idx       [T*k]  int32 in [0, E)
+ *   expert_offsets [E+1]  int32 out
+ *   sorted_pair    [T*k]  int32 out
+ *   pair_row       [T*k]  int32 out
+ *   Limits: 1 <= E <= 1024, 0 <= T*k <= 1<<24.  An id outside [0,E) sets
+ *   MOE_DEV_BAD_EXPERT and that pair is left out.
+ */
+int moe_permute(const int32_t *topk_idx, int T, int k, int E,
+                int32_t *expert_offsets, int32_t *sorted_pair,
+                int32_t *pair_row, moe_stream_t stream);
+
+/*
+ * mxfp4_moe_ffn -- SwiGLU FFN of every permuted pair over MXFP4 experts.
+ *   The experts hold OCP MXFP4 weights while the rest of the model keeps
+ *   higher precision ([P1] "接受率预测与动态回退机制"; [P3] "FP4 Expert 量化";
+ *   [P4] "第一层：FP4 选择性量化").  Weight format [OCP]: 4-bit E2M1 codes,
+ *   two per byte (element 2j in the low nibble), one E8M0 scale byte
+ *   (value 2^(s-127)) per 32 consecutive elements of a row.
+ *     w13_codes  [E, 2I, H/2]  uint8   rows 0..I-1 gate, I..2I-1 up
+ *     w13_scales [E, 2I, H/32] uint8
+ *     w2_codes   [E, H, I/2]   uint8   down projection
+ *     w2_scales  [E, H, I/32]  uint8
+ *   For sorted row r of expert e (token t = sorted_pair[r] / k):
+ *     g = x[t] . Wg^T, u = x[t] . Wu^T   (float accumulation over the exactly
+ *     dequantised weights), h = bf16(silu(g) * u), y[r] = h . Wd^T (float).
+ *   x              [T, H]     bf16
+ *   expert_offsets [E+1], sorted_pair [T*k]  from moe_permute
+ *   y              [T*k, H]   float out, sorted-row order
+ *   workspace      device scratch of at least
+ *                  mxfp4_moe_ffn_workspace_bytes(T, k, H, I) bytes, 256-byte
+ *                  aligned; its contents on entry do not matter.
+ *   Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
+ *   The kernel variant is chosen from the average number of rows per expert
+ *   (see mxfp4_moe_ffn_variant).
+ */
+size_t mxfp4_moe_ffn_workspace_bytes(int T, int k, int H, int I);
+
+int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
+                  const uint8_t *w13_codes, const uint8_t *w13_scales,
+                  const uint8_t *w2_codes, const uint8_t *w2_scales,
+                  const int32_t *expert_offsets, const int32_t *sorted_pair,
+                  float *y, void *workspace, size_t workspace_bytes,
+                  moe_stream_t stream);
+
+/* Kernel variants of mxfp4_moe_ffn. */
+enum {
+  MOE_FFN_AUTO = 0,   /* pick by T*k / E                                  */
+  MOE_FFN_FMA = 1,    /* dequantise to registers, float FMA (small N)     */
+  MOE_FFN_TENSOR = 2  /* tcgen05 block-scaled MMA, TMEM accumulators      */
+};
+
+/* Same contract as mxfp4_moe_ffn with an explicit kernel variant. */
+int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
+                          const uint8_t *w13_codes, const uint8_t *w13_scales,
+                          const uint8_t *w2_codes, const uint8_t *w2_scales,
+                          const int32_t *expert_offsets,
+                          const int32_t *sorted_pair, float *y, void *workspace,
+                          size_t workspace_bytes, int variant,
+                          moe_stream_t stream);
+
+/* The bf16 SwiGLU outputs h [T*k, I] (sorted-row order) that the last
+ * mxfp4_moe_ffn call left at the start of its workspace. */
+const uint16_t *mxfp4_moe_ffn_workspace_h(const void *workspace);
+
+/*
+ * moe_combine -- weighted sum of each token's k expert outputs.
+ *   out[t] = bf16( sum_{j<k} topk_w[t,j] * y[pair_row[t*k+j]] + residual[t] )
+ *   in float, slots summed in order j = 0..k-1, residual added last.
+ *   y [T*k, H] float, pair_row [T*k], topk_w [T, k] float,
+ *   residual [T, H] bf16 or NULL, out [T, H] bf16 (may alias residual).
+ */
+int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w,
+                int T, int k, int H, const uint16_t *residual, uint16_t *out,
+                moe_stream_t stream);
+
+/*
+ * moe_rms_norm -- parameter-free RMSNorm of bf16 rows (stacked layers).
+ *   out[t] = bf16( x[t] / sqrt(mean_c x[t,c]^2 + eps) ), float arithmetic.
+ *   The pages do not describe the layer stack; a pre-norm keeps stacked
+ *   synthetic layers finite (each MXFP4 expert layer scales its input by
+ *   ~1e8 at the configured scale range).  x, out [T, H] bf16, may alias.
+ */
+int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
+                 moe_stream_t stream);
+
+/*
+ * block_accept_greedy -- greedy prefix acceptance of S drafted blocks.
+ *   Tokens the target confirms are kept; from the first wrong draft token
+ *   on the target takes over ([P2] "二、投机解码").  Row i of logits checks
+ *   draft[i]; accept_len = the largest a such that argmax(logits[s,i]) ==
+ *   draft[s,i] for all i < a (argmax ties to the lowest token id);
+ *   next_token = argmax(logits[s, a]) if a < K, else -1.
+ *   logits [S, K, V] float, draft [S, K] int32,
+ *   accept_len [S] int32 out, next_token [S] int32 out.
+ *   Limits: 1 <= K <= 32, 1 <= V < 2^31.
+ */
+int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
+                        int V, int32_t *accept_len, int32_t *next_token,
+                        moe_stream_t stream);
+
+/*
+ * block_accept_rejection -- speculative rejection sampling of S blocks.
+ *   Verify by rejection sampling ([P3] "数据流概览"), lossless in the sense
+ *   that the output follows the target distribution ([P2] "六、效果如何").
+ *   Draft x_i is accepted iff double(u_accept[s,i]) * double(q[s,i,x_i]) <
+ *   double(p[s,i,x_i]) (= u < min(1, p/q), exactly).  At the first rejected
+ *   row a the token is drawn from max(0, p - q): r_v = max(0, p_v - q_v) in
+ *   float, R_v = floor(r_v * 2^40) (integer), m = floor(sum(R) * U / 2^24)
+ *   with U = u_resample[s] * 2^24, next_token = least v with
+ *   R_0 + .. + R_v > m; if sum(R) == 0 the same draw uses floor(p_v * 2^40).
+ *   All K accepted -> next_token = -1.
+ *   p, q [S, K, V] float probabilities; draft [S, K] int32;
+ *   u_accept [S, K], u_resample [S] float uniforms in [0,1), multiples of
+ *   2^-24; accept_len [S], next_token [S] int32 out.
+ *   Limits: 1 <= K <= 32, 1 <= V <= 2^24.
+ */
+int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
+                           const float *u_accept, const float *u_resample,
+                           int S, int K, int V, int32_t *accept_len,
+                           int32_t *next_token, moe_stream_t stream);
+
+/*
+ * moe_get_device_status -- synchronise `stream`, then report the sticky
+ * device status word of the current device: returns MOE_OK if it is clear,
+ * MOE_ERR_DEVICE if set (detail in *detail, may be NULL), MOE_ERR_CUDA on a
+ * CUDA failure.  moe_clear_device_status resets it (enqueued on `stream`).
+ */
+int moe_get_device_status(moe_stream_t stream, int *detail);
+int moe_clear_device_status(moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_MOE_H */

@@ -1,0 +1,14 @@
+"""MXFP4 MoE block-verify on B200: a C-ABI CUDA library with a thin binding.
+
+The six calls of the verify step -- moe_route_topk, moe_permute,
+mxfp4_moe_ffn, moe_combine, block_accept_greedy, block_accept_rejection --
+plus moe_rms_norm for stacked layers, all run as hand-written sm_100a
+kernels in libmxfp4_moe.so (see include/mxfp4_moe.h).  Importing the package
+does not load the library; the first call does, and raises if it is missing.
+"""
+from ._lib import (  # noqa: F401
+    FFN_AUTO, FFN_FMA, FFN_TENSOR, MoeError, alloc_workspace, block_accept_greedy,
+    block_accept_rejection, lib, moe_clear_device_status, moe_combine, moe_get_device_status,
+    moe_permute, moe_rms_norm, moe_route_topk, mxfp4_moe_ffn, mxfp4_moe_ffn_workspace_bytes,
+    workspace_h,
+)

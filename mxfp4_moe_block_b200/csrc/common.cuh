@@ -1,0 +1,88 @@
+// common.cuh -- device helpers shared by the kernels of the MXFP4 MoE
+// block-verify library (sm_100a).  Built as one translation unit with
+// mxfp4_moe.cu, so __device__ globals here are visible to every kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/mxfp4_moe.h"
+
+namespace moe {
+
+// Sticky device status word: the first error detail wins.
+__device__ int g_status;
+
+__device__ __forceinline__ void raise_status(int detail) {
+  atomicCAS(&g_status, 0, detail);
+}
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// bf16 bit patterns packed two per 32-bit word -> float.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t *>(&b);
+}
+
+// E8M0 scale byte -> 2^(e-127) as float (0 -> 2^-127, a subnormal; 255 -> NaN).
+__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
+  if (e == 0u) return __uint_as_float(0x00400000u);
+  if (e == 255u) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float(e << 23);
+}
+
+// Two E2M1 codes of one byte (low nibble = even element) -> two floats, exact.
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
+  __half2_raw r = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xffu), __NV_E2M1);
+  return __half22float2(*reinterpret_cast<__half2 *>(&r));
+}
+
+// 16-byte streaming load that bypasses L1 (weights are read exactly once).
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ld_nc16(const void *p) {
+  return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+  return v;
+}
+
+// (value, index) argmax order: larger value first, then the lower index.
+// idx < 0 marks "no candidate".
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return bi < 0 || (i >= 0 && (v > bv || (v == bv && i < bi)));
+}
+
+__device__ __forceinline__ void warp_argmax(float &v, int &i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float ov = __shfl_xor_sync(FULL, v, o);
+    int oi = __shfl_xor_sync(FULL, i, o);
+    if (better(ov, oi, v, i)) { v = ov; i = oi; }
+  }
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+}  // namespace moe

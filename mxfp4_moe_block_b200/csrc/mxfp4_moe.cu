@@ -1,0 +1,284 @@
+// mxfp4_moe.cu -- the C ABI of include/mxfp4_moe.h: argument checks, kernel
+// choice and launches.  Every kernel of the library is compiled into this one
+// translation unit (the .cuh files), for sm_100a.
+#include <cstdio>
+#include <cstring>
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "route_permute.cuh"
+#include "ffn_fma.cuh"
+#include "ffn_tc.cuh"
+#include "combine.cuh"
+#include "accept.cuh"
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device(int *dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+const DeviceInfo *device_info() {
+  int dev;
+  if (current_device(&dev) != MOE_OK) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return nullptr;
+    d.ready = true;
+  }
+  return &d;
+}
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "mxfp4_moe: launch failed: %s\n", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or variant";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MOE_ERR_DEVICE: return "device status word set";
+    default: return "unknown status";
+  }
+}
+
+int moe_version(void) { return 10000; }
+
+// ------------------------------------------------------------------ route --
+int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
+                   float *topk_w, moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  const dim3 block(128), grid((unsigned)((T + 3) / 4));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (E <= 32) route_topk_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 64) route_topk_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 128) route_topk_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 256) route_topk_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  else if (E <= 512) route_topk_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  else route_topk_kernel<32><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- permute --
+int moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *expert_offsets,
+                int32_t *sorted_pair, int32_t *pair_row, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  const long long P = (long long)T * k;
+  if (P > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+  if (P > 0 && (!topk_idx || !sorted_pair || !pair_row)) return MOE_ERR_INVALID_ARG;
+  const size_t smem = (size_t)33 * E * sizeof(int);
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         33 * 1024 * (int)sizeof(int));
+  });
+  permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(topk_idx, (int)P, E, expert_offsets,
+                                                           sorted_pair, pair_row);
+  return launch_status();
+}
+
+// -------------------------------------------------------------------- FFN --
+// Workspace layout (each part 256-byte aligned): h bf16 [P, I] first (the
+// documented accessor), then x as float [T, H], h as float [P, I], then the
+// tensor-core variant's operands.
+struct WsLayout {
+  size_t h, x32, h32, tc, total;
+};
+
+static WsLayout ws_layout(int T, int k, int H, int I) {
+  const size_t P = (size_t)T * k;
+  WsLayout w;
+  size_t o = 0;
+  w.h = o;   o += align256(P * I * sizeof(uint16_t));
+  w.x32 = o; o += align256((size_t)T * H * sizeof(float));
+  w.h32 = o; o += align256(P * I * sizeof(float));
+  w.tc = o;  o += tc_workspace_bytes(P, H, I);
+  w.total = o < 256 ? 256 : o;
+  return w;
+}
+
+size_t mxfp4_moe_ffn_workspace_bytes(int T, int k, int H, int I) {
+  if (T < 0 || k < 1 || H < 0 || I < 0) return 0;
+  return ws_layout(T, k, H, I).total;
+}
+
+const uint16_t *mxfp4_moe_ffn_workspace_h(const void *workspace) {
+  return reinterpret_cast<const uint16_t *>(workspace);
+}
+
+int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
+                          const uint8_t *w13_codes, const uint8_t *w13_scales,
+                          const uint8_t *w2_codes, const uint8_t *w2_scales,
+                          const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
+                          void *workspace, size_t workspace_bytes, int variant,
+                          moe_stream_t stream) {
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (variant < MOE_FFN_AUTO || variant > MOE_FFN_TENSOR) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !expert_offsets ||
+      !sorted_pair || !y || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < mxfp4_moe_ffn_workspace_bytes(T, k, H, I) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MOE_ERR_WORKSPACE;
+  const DeviceInfo *dev = device_info();
+  if (!dev) return MOE_ERR_CUDA;
+  const size_t P = (size_t)T * k;
+  if (variant == MOE_FFN_AUTO) variant = tc_prefer(P, E) ? MOE_FFN_TENSOR : MOE_FFN_FMA;
+
+  const WsLayout wl = ws_layout(T, k, H, I);
+  uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+  FfnArgs a{x, T, H, I, E, k, w13_codes, w13_scales, w2_codes, w2_scales,
+            expert_offsets, sorted_pair, reinterpret_cast<uint16_t *>(ws + wl.h), y,
+            reinterpret_cast<float *>(ws + wl.x32), reinterpret_cast<float *>(ws + wl.h32)};
+  cudaStream_t s = (cudaStream_t)stream;
+  if (variant == MOE_FFN_TENSOR) return tc_ffn(a, ws + wl.tc, dev->sms, s);
+  const size_t n8 = (size_t)T * H / 8;
+  x_to_f32_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8), 256, 0, s>>>(
+      x, n8, a.x32);
+  int st = launch_status();
+  if (st != MOE_OK) return st;
+  ffn1_fma_kernel<4><<<dev->sms, FMA_THREADS, 0, s>>>(a);
+  st = launch_status();
+  if (st != MOE_OK) return st;
+  ffn2_fma_kernel<8><<<dev->sms, FMA_THREADS, 0, s>>>(a);
+  return launch_status();
+}
+
+int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
+                  const uint8_t *w13_codes, const uint8_t *w13_scales,
+                  const uint8_t *w2_codes, const uint8_t *w2_scales,
+                  const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
+                  void *workspace, size_t workspace_bytes, moe_stream_t stream) {
+  return mxfp4_moe_ffn_variant(x, T, H, I, E, k, w13_codes, w13_scales, w2_codes, w2_scales,
+                               expert_offsets, sorted_pair, y, workspace, workspace_bytes,
+                               MOE_FFN_AUTO, stream);
+}
+
+// ---------------------------------------------------------------- combine --
+int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w, int T, int k,
+                int H, const uint16_t *residual, uint16_t *out, moe_stream_t stream) {
+  if (T < 0 || k < 1 || k > 32 || H <= 0 || H % 8) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !pair_row || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  const dim3 grid((unsigned)T, (unsigned)((H + 1023) / 1024));
+  combine_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(y, pair_row, topk_w, T, k, H, residual,
+                                                         out);
+  return launch_status();
+}
+
+int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
+                 moe_stream_t stream) {
+  if (T < 0 || H <= 0 || H % 8 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !out) return MOE_ERR_INVALID_ARG;
+  rms_norm_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(x, T, H, eps, out);
+  return launch_status();
+}
+
+// ----------------------------------------------------------------- accept --
+int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K, int V,
+                        int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  if (S < 0 || K < 1 || K > 32 || V < 1) return MOE_ERR_INVALID_ARG;
+  if (S == 0) return MOE_OK;
+  if (!logits || !draft || !accept_len || !next_token) return MOE_ERR_INVALID_ARG;
+  if (S > 65535) return MOE_ERR_UNSUPPORTED;
+  const int per_cta = 4 * GREEDY_THREADS;           // elements per CTA and pass
+  int csize = GREEDY_CLUSTER;
+  while (csize > 1 && (long long)V < (long long)csize * per_cta) csize >>= 1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(greedy_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  });
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize, S, 1);
+  cfg.blockDim = dim3(GREEDY_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t err =
+      cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, accept_len, next_token);
+  if (err != cudaSuccess) {
+    fprintf(stderr, "mxfp4_moe: cluster launch failed: %s\n", cudaGetErrorString(err));
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
+                           const float *u_accept, const float *u_resample, int S, int K, int V,
+                           int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  if (S < 0 || K < 1 || K > 32 || V < 1 || V > (1 << 24)) return MOE_ERR_INVALID_ARG;
+  if (S == 0) return MOE_OK;
+  if (!p || !q || !draft || !u_accept || !u_resample || !accept_len || !next_token)
+    return MOE_ERR_INVALID_ARG;
+  if (S > (1 << 30)) return MOE_ERR_UNSUPPORTED;
+  int threads = ((V + 31) / 32) * 32;
+  if (threads > 1024) threads = 1024;
+  rejection_kernel<<<S, threads, 0, (cudaStream_t)stream>>>(p, q, draft, u_accept, u_resample,
+                                                            S, K, V, accept_len, next_token);
+  return launch_status();
+}
+
+// ----------------------------------------------------------------- status --
+int moe_get_device_status(moe_stream_t stream, int *detail) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (detail) *detail = v;
+  return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+int moe_clear_device_status(moe_stream_t stream) {
+  void *addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_status) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(addr, 0, sizeof(int), (cudaStream_t)stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,152 @@
+// route_permute.cuh -- top-k routing and the stable grouping of
+// (token, slot) pairs by expert.
+//
+// Routing: each token activates a few experts ("mimo-tilert-1000tps-trillion-
+// parameter-inference", section "万亿参数推理为什么特别难"); the selection
+// rule (descending logit, ties to the lowest index) and the softmax over the
+// selected logits are the library's stated reading, the pages being silent.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// One warp per token.  Lane l holds logits l, l+32, ... (PER per lane).
+// k rounds of a warp argmax pick the experts in rank order; the winner's
+// owner lane marks it taken.  Weights: softmax of the selected logits in
+// double, summed in slot order, rounded once to float.
+template <int PER>
+__global__ void __launch_bounds__(128)
+route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                  int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const float *row = logits + (size_t)t * E;
+  float v[PER];
+  unsigned taken = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __ldg(row + e) : 0.f;
+    if (e >= E) taken |= 1u << i;
+  }
+  float my_v = 0.f;
+  int my_i = -1;
+  for (int r = 0; r < k; ++r) {
+    float bv = 0.f;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      if (!((taken >> i) & 1u) && better(v[i], lane + 32 * i, bv, bi)) {
+        bv = v[i];
+        bi = lane + 32 * i;
+      }
+    }
+    warp_argmax(bv, bi);
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == r) { my_v = bv; my_i = bi; }
+  }
+  const float vmax = __shfl_sync(FULL, my_v, 0);
+  const double ex = (lane < k) ? exp((double)my_v - (double)vmax) : 0.0;
+  double sum = 0.0;
+  for (int j = 0; j < k; ++j) sum += __shfl_sync(FULL, ex, j);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_i;
+    topk_w[(size_t)t * k + lane] = (float)(ex / sum);
+  }
+}
+
+// Stable counting sort of P = T*k pairs by expert in one CTA of 1024 threads.
+// Warp w owns the contiguous pair range [w*seg, (w+1)*seg).
+//   pass A: per-warp, per-expert running counts; each pair's rank inside its
+//           warp's range (lanes with equal experts found by __match_any_sync)
+//           is parked in pair_row[p];
+//   pass B: per expert, exclusive prefix over warps; block scan of the
+//           per-expert totals gives expert_offsets;
+//   pass C: pos = offset[e] + warp_base[w][e] + local rank.
+// Dynamic shared memory: 32*E counters + E offsets (ints).
+__global__ void __launch_bounds__(1024)
+permute_kernel(const int32_t *__restrict__ topk_idx, int P, int E,
+               int32_t *__restrict__ expert_offsets,
+               int32_t *__restrict__ sorted_pair, int32_t *__restrict__ pair_row) {
+  extern __shared__ int smem[];
+  int *cnt = smem;             // [32][E]
+  int *offs = smem + 32 * E;   // [E]
+  __shared__ int warp_tot[32];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int seg = (P + 31) / 32;
+  const int p0 = min(P, w * seg), p1 = min(P, p0 + seg);
+
+  for (int e = lane; e < E; e += 32) cnt[w * E + e] = 0;
+  __syncwarp();
+  // pass A
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    int e = -1;
+    if (p < p1) {
+      e = topk_idx[p];
+      if (e < 0 || e >= E) { raise_status(MOE_DEV_BAD_EXPERT); e = -1; }
+    }
+    const unsigned same = __match_any_sync(FULL, e);
+    int before = 0;
+    if (e >= 0) before = cnt[w * E + e];
+    __syncwarp();
+    if (e >= 0) {
+      pair_row[p] = before + __popc(same & lanemask_lt());
+      if ((same & lanemask_lt()) == 0) cnt[w * E + e] = before + __popc(same);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  // pass B: per expert, exclusive prefix over warps (E <= 1024, checked on
+  // the host, so thread e owns expert e); then a block scan of the totals.
+  const int e = threadIdx.x;
+  int tot = 0;
+  if (e < E) {
+    for (int ww = 0; ww < 32; ++ww) {
+      const int c = cnt[ww * E + e];
+      cnt[ww * E + e] = tot;
+      tot += c;
+    }
+  }
+  int x = tot;  // inclusive scan of tot over the block
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(FULL, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int s = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(FULL, s, o);
+      if (lane >= o) s += y;
+    }
+    warp_tot[lane] = s;  // inclusive over warps
+  }
+  __syncthreads();
+  const int incl = x + (w > 0 ? warp_tot[w - 1] : 0);
+  if (e < E) {
+    offs[e] = incl - tot;
+    expert_offsets[e] = incl - tot;
+    if (e == E - 1) expert_offsets[E] = incl;
+  }
+  __syncthreads();
+  // pass C
+  for (int base = p0; base < p1; base += 32) {
+    const int p = base + lane;
+    if (p < p1) {
+      const int e = topk_idx[p];
+      if (e >= 0 && e < E) {
+        const int pos = offs[e] + cnt[w * E + e] + pair_row[p];
+        sorted_pair[pos] = p;
+        pair_row[p] = pos;
+      }
+    }
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,53 @@
+"""The C-ABI library loads on a machine without a GPU and exports every
+function include/*.h declares; the binding declares the same set."""
+import glob
+import os
+import re
+
+import pytest
+
+from mxfp4_moe_block_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h, encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            if m.group(1) not in ("if", "while", "for", "return"):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def library():
+    build.build()
+    return _lib.lib()
+
+
+def test_header_declares_the_six_calls():
+    d = declared_functions()
+    for n in ("moe_route_topk", "moe_permute", "mxfp4_moe_ffn", "moe_combine",
+              "block_accept_greedy", "block_accept_rejection"):
+        assert n in d
+
+
+def test_every_declared_symbol_is_exported(library):
+    for n in declared_functions():
+        assert hasattr(library, n), n
+
+
+def test_binding_covers_the_header():
+    assert set(declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_host_only_calls(library):
+    assert library.moe_version() == 10000
+    assert library.moe_status_string(4) == b"workspace too small or misaligned"
+    assert library.mxfp4_moe_ffn_workspace_bytes(8, 8, 7168, 2048) >= 64 * 2048 * 2
+    # argument checks return before any CUDA call
+    assert library.moe_route_topk(None, 4, 8, 9, None, None, None) == 1
+    assert library.block_accept_greedy(None, None, 1, 0, 10, None, None, None) == 1

@@ -1,0 +1,412 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on
+the same seeded inputs, for the five workload shapes and the edge cases.
+
+Bit-exact: routing indices, permutation, acceptance.  Routing weights: equal
+floats except at a float rounding midpoint.  FFN, combine and the stacked
+layers: rel-L2 <= 2e-3 and max-abs <= 1e-2 * max|ref|.  Full-size shapes
+compare sampled experts (every row of each sampled expert), which the oracle
+computes one by one; the tiny shape compares everything.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_moe_block_b200 as mm
+from mxfp4_moe_block_b200 import synth
+from oracle import accept as oacc
+from oracle import moe as omoe
+from oracle import mxfp4 as omx
+
+from gpu_helpers import (Layer, assert_ffn_close, assert_route_weights, bf16_tensor,
+                         bf16_to_f64)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ALL = ["tiny", "batch1", "serving", "dflash16", "multilayer"]
+
+
+@pytest.fixture(autouse=True)
+def clean_status():
+    mm.moe_clear_device_status()
+    yield
+
+
+def _route_permute(L, sh):
+    idx, w = mm.moe_route_topk(L.logits, sh.k)
+    off, sp, pr = mm.moe_permute(idx, sh.E)
+    return idx, w, off, sp, pr
+
+
+# ------------------------------------------------------- routing, permute --
+
+@pytest.mark.parametrize("name", ALL)
+def test_route_permute_bit_exact(name):
+    sh = synth.SHAPES[name]
+    for layer in range(min(sh.layers, 2)):
+        L = Layer(sh, layer, DEV, with_weights=False)
+        idx, w, off, sp, pr = _route_permute(L, sh)
+        ridx, _, rw64 = omoe.route_topk(L.logits_np, sh.k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert_route_weights(w.cpu().numpy(), rw64)
+        roff, rsp, rpr = omoe.permute(ridx, sh.E)
+        assert np.array_equal(off.cpu().numpy(), roff)
+        assert np.array_equal(sp.cpu().numpy(), rsp)
+        assert np.array_equal(pr.cpu().numpy(), rpr)
+        assert mm.moe_get_device_status() == (0, 0)
+
+
+def test_route_ties_signed_zero_and_max_sizes():
+    rng = np.random.default_rng(5)
+    for T, E, k in [(33, 1, 1), (64, 5, 5), (100, 8, 3), (17, 1024, 32), (40, 300, 7)]:
+        pool = np.array([-0.0, 0.0, 1.0, -2.5, 3.0], np.float32)
+        l = pool[rng.integers(0, 5, (T, E))]
+        idx, w = mm.moe_route_topk(torch.from_numpy(l).to(DEV), k)
+        ridx, _, rw64 = omoe.route_topk(l, k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert_route_weights(w.cpu().numpy(), rw64)
+
+
+def test_permute_large_properties():
+    """P = 2**19 pairs over 1024 experts, against numpy's stable argsort."""
+    T, k, E = 65536, 8, 1024
+    idx = synth.int_range_np(synth.stream_key(7, "router"), 0, T * k, 0, E - 1)
+    idx = idx.astype(np.int32).reshape(T, k)
+    off, sp, pr = mm.moe_permute(torch.from_numpy(idx).to(DEV), E)
+    want = np.argsort(idx.reshape(-1), kind="stable")
+    assert np.array_equal(sp.cpu().numpy(), want)
+    assert np.array_equal(pr.cpu().numpy()[want], np.arange(T * k))
+    counts = np.bincount(idx.reshape(-1), minlength=E)
+    assert np.array_equal(off.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
+
+
+def test_permute_empty_and_bad_expert():
+    off, sp, pr = mm.moe_permute(torch.zeros((0, 2), dtype=torch.int32, device=DEV), 4)
+    assert off.cpu().tolist() == [0] * 5
+    bad = torch.tensor([[0, 9], [1, 2]], dtype=torch.int32, device=DEV)
+    mm.moe_permute(bad, 4)
+    assert mm.moe_get_device_status() == (mm._lib.MOE_OK + 5, 1)
+
+
+# -------------------------------------------------------------- expert FFN --
+
+def _sample_experts(off, n=4):
+    cnt = np.diff(off)
+    act = np.nonzero(cnt)[0]
+    if len(act) <= n:
+        return list(act)
+    pick = {int(act[np.argmax(cnt[act])])}
+    if n > 1:
+        pick.add(int(act[np.argmin(cnt[act])]))
+    rest = [int(e) for e in act if int(e) not in pick]
+    step = max(1, len(rest) // (n - len(pick) + 1))
+    for e in rest[step // 2::step]:
+        if len(pick) >= n:
+            break
+        pick.add(e)
+    return sorted(pick)
+
+
+def _ffn_check(name, layer, variant, n_experts=4):
+    sh = synth.SHAPES[name]
+    L = Layer(sh, layer, DEV)
+    idx, w, off, sp, pr = _route_permute(L, sh)
+    y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=variant)
+    torch.cuda.synchronize()
+    ridx, _, _ = omoe.route_topk(L.logits_np, sh.k)
+    roff, rsp, _ = omoe.permute(ridx, sh.E)
+    assert np.array_equal(off.cpu().numpy(), roff)
+    x64 = L.x_f64()
+    yg = y.cpu().numpy()
+    hg = bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I))
+    if name == "tiny":
+        h_ref, y_ref = omoe.moe_ffn(x64, sh.k, sh.I, L.oracle_weights, roff, rsp)
+        eh = assert_ffn_close(hg, h_ref, "h")
+        ey = assert_ffn_close(yg, y_ref, "y")
+        print(f"[ffn {name} variant {variant}] h rel-L2 {eh[0]:.2e}  y rel-L2 {ey[0]:.2e}")
+        return
+    for e in _sample_experts(roff, n_experts):
+        r0, r1 = int(roff[e]), int(roff[e + 1])
+        toks = rsp[r0:r1] // sh.k
+        he, ye = omoe.expert_ffn(x64[toks], *L.oracle_weights(e), sh.I)
+        eh = assert_ffn_close(hg[r0:r1], he, f"h expert {e}")
+        ey = assert_ffn_close(yg[r0:r1], ye, f"y expert {e}")
+        print(f"[ffn {name} variant {variant}] expert {e} rows {r1 - r0}: "
+              f"h rel-L2 {eh[0]:.2e}  y rel-L2 {ey[0]:.2e}")
+
+
+@pytest.mark.parametrize("name", ALL)
+def test_ffn_fma(name):
+    _ffn_check(name, 0, mm.FFN_FMA)
+
+
+@pytest.mark.parametrize("name", ["batch1", "serving", "dflash16", "multilayer"])
+def test_ffn_tensor(name):
+    _ffn_check(name, 0, mm.FFN_TENSOR)
+
+
+def test_ffn_tensor_small_shapes_and_bn_classes():
+    """tcgen05 path on small shapes: one expert with many rows (several B
+    tiles, a ragged last one) and every B-tile width class."""
+    for K, E, k in [(1, 4, 1), (37, 4, 1), (64, 2, 2), (200, 2, 1), (8, 64, 8)]:
+        sh = synth.Shape("tcs", H=512, I=256, E=E, k=k, S=1, K=K, V=64, seed=20 + K)
+        L = Layer(sh, 0, DEV)
+        idx, w, off, sp, pr = _route_permute(L, sh)
+        y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=mm.FFN_TENSOR)
+        ridx, _, _ = omoe.route_topk(L.logits_np, sh.k)
+        roff, rsp, _ = omoe.permute(ridx, sh.E)
+        h_ref, y_ref = omoe.moe_ffn(L.x_f64(), sh.k, sh.I, L.oracle_weights, roff, rsp)
+        assert_ffn_close(bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I)), h_ref, f"h K={K}")
+        assert_ffn_close(y.cpu().numpy(), y_ref, f"y K={K}")
+        assert mm.moe_get_device_status() == (0, 0)
+
+
+def test_ffn_one_expert_many_tokens():
+    """Every token on one expert (37 rows: several passes and a ragged one)."""
+    sh = synth.Shape("one", H=256, I=128, E=4, k=1, S=1, K=37, V=64, seed=11)
+    L = Layer(sh, 0, DEV)
+    L.logits_np[:, 2] += 100.0
+    L.logits = torch.from_numpy(L.logits_np).to(DEV)
+    for variant in (mm.FFN_FMA,):
+        idx, w, off, sp, pr = _route_permute(L, sh)
+        assert np.diff(off.cpu().numpy()).tolist() == [0, 0, 37, 0]
+        y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=variant)
+        he, ye = omoe.expert_ffn(L.x_f64()[sp.cpu().numpy()], *L.oracle_weights(2), sh.I)
+        assert_ffn_close(y.cpu().numpy(), ye, "y")
+
+
+def test_ffn_empty_batch():
+    sh = synth.SHAPES["tiny"]
+    L = Layer(sh, 0, DEV)
+    x = L.x[:0]
+    off = torch.zeros(sh.E + 1, dtype=torch.int32, device=DEV)
+    sp = torch.zeros(0, dtype=torch.int32, device=DEV)
+    y, _ = mm.mxfp4_moe_ffn(x, sh.k, *L.w, off, sp)
+    assert y.shape == (0, sh.H)
+
+
+# ----------------------------------------------------------- combine, norm --
+
+@pytest.mark.parametrize("name", ["tiny", "batch1", "serving", "dflash16"])
+def test_combine(name):
+    sh = synth.SHAPES[name]
+    T, k, H, P = sh.T, sh.k, sh.H, sh.P
+    key = synth.stream_key(sh.seed + 50, "x")
+    y = (1e3 * synth.normal_np(key, 0, P * H)).astype(np.float32).reshape(P, H)
+    perm = np.argsort(synth.hash_np(key, 0, P)).astype(np.int32)
+    w = synth.u24_np(key, 0, T * k).reshape(T, k)
+    res_bits = synth.x_bf16_bits(sh, 3)
+    out_g = mm.moe_combine(torch.from_numpy(y).to(DEV), torch.from_numpy(perm).to(DEV),
+                           torch.from_numpy(w).to(DEV), residual=bf16_tensor(res_bits, DEV))
+    res = synth.bf16_bits_to_f32(res_bits).astype(np.float64)
+    out_r, acc_r = omoe.combine(y.astype(np.float64), perm, w, res)
+    assert_ffn_close(bf16_to_f64(out_g), out_r, "combine")
+    # in place: out aliases residual
+    rt = bf16_tensor(res_bits, DEV)
+    mm.moe_combine(torch.from_numpy(y).to(DEV), torch.from_numpy(perm).to(DEV),
+                   torch.from_numpy(w).to(DEV), residual=rt, out=rt)
+    assert torch.equal(rt, out_g)
+
+
+def test_rms_norm():
+    sh = synth.SHAPES["multilayer"]
+    bits = synth.x_bf16_bits(sh, 5)
+    x = synth.bf16_bits_to_f32(bits).astype(np.float64) * 3e7
+    xb = torch.from_numpy(x.astype(np.float32)).to(DEV).to(torch.bfloat16)
+    got = bf16_to_f64(mm.moe_rms_norm(xb))
+    ref = omoe.rms_norm(bf16_to_f64(xb))
+    assert_ffn_close(got, ref, "rms_norm")
+
+
+# --------------------------------------------------------------- acceptance --
+
+@pytest.mark.parametrize("name", ["tiny", "batch1", "serving", "multilayer"])
+def test_greedy_bit_exact(name):
+    sh = synth.SHAPES[name]
+    lg = synth.block_logits(sh)
+    d = synth.greedy_drafts(sh, lg)
+    acc, nxt = mm.block_accept_greedy(torch.from_numpy(lg).to(DEV), torch.from_numpy(d).to(DEV))
+    racc, rnxt = oacc.greedy(lg, d)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert np.array_equal(nxt.cpu().numpy(), rnxt)
+
+
+def test_greedy_edges():
+    rng = np.random.default_rng(9)
+    for S, K, V in [(3, 1, 1), (5, 32, 1001), (2, 8, 7), (4, 3, 5000)]:
+        lg = rng.integers(-3, 3, (S, K, V)).astype(np.float32)       # many ties
+        am = lg.argmax(-1).astype(np.int32)
+        for d in (am, np.where(rng.random((S, K)) < 0.3, (am + 1) % V, am).astype(np.int32)):
+            acc, nxt = mm.block_accept_greedy(torch.from_numpy(lg).to(DEV), torch.from_numpy(d).to(DEV))
+            racc, rnxt = oacc.greedy(lg, d)
+            assert np.array_equal(acc.cpu().numpy(), racc)
+            assert np.array_equal(nxt.cpu().numpy(), rnxt)
+
+
+@pytest.mark.parametrize("name", ["dflash16", "multilayer"])
+def test_rejection_bit_exact(name):
+    sh = synth.SHAPES[name]
+    ri = synth.rejection_inputs(sh)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    acc, nxt = mm.block_accept_rejection(t(ri.p), t(ri.q), t(ri.draft), t(ri.u_accept),
+                                         t(ri.u_resample))
+    racc, rnxt = oacc.rejection(ri.p, ri.q, ri.draft, ri.u_accept, ri.u_resample)
+    assert np.array_equal(acc.cpu().numpy(), racc)
+    assert np.array_equal(nxt.cpu().numpy(), rnxt)
+    assert mm.moe_get_device_status() == (0, 0)
+
+
+def test_rejection_edges():
+    V = 3000
+    rng = np.random.default_rng(3)
+    p = rng.random((6, 4, V)).astype(np.float32)
+    p /= p.sum(-1, keepdims=True)
+    q = p.copy()
+    q[1] = np.roll(p[1], 7, axis=-1)           # independent-ish rows
+    q[2, 0] = 0.0
+    q[2, 0, 5] = 1.0                            # residual = p except at token 5
+    d = rng.integers(0, V, (6, 4)).astype(np.int32)
+    ua = (rng.integers(0, 2 ** 24, (6, 4)) * 2.0 ** -24).astype(np.float32)
+    ur = (rng.integers(0, 2 ** 24, 6) * 2.0 ** -24).astype(np.float32)
+    ua[3] = np.float32(1 - 2.0 ** -24)
+    q[3] = np.where(np.arange(V) == d[3, 0, None], 0.0, q[3])   # q(x)=0 -> accept
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    acc, nxt = mm.block_accept_rejection(t(p), t(q), t(d), t(ua), t(ur))
+    racc, rnxt = oacc.rejection(p, q, d, ua, ur)
+    assert np.array_equal(acc.cpu().numpy(), racc) and np.array_equal(nxt.cpu().numpy(), rnxt)
+    assert racc[0] == 4 and racc[3] >= 1
+
+
+def test_rejection_bad_token_sets_status():
+    p = torch.full((1, 1, 8), 0.125, device=DEV)
+    d = torch.tensor([[8]], dtype=torch.int32, device=DEV)
+    ua = torch.zeros((1, 1), device=DEV)
+    ur = torch.zeros(1, device=DEV)
+    mm.block_accept_rejection(p, p, d, ua, ur)
+    assert mm.moe_get_device_status() == (5, 3)
+
+
+def test_rejection_lossless_chi2_on_gpu():
+    """Emitted-token marginal == target p over 10**6 seeded single-token
+    blocks (chi-square, 15 dof, p >= 0.001), as for the oracle."""
+    n, V, seed = 1_000_000, 16, 77
+    zp = synth.normal_np(synth.stream_key(seed, "p_logits"), 0, V)
+    zq = synth.normal_np(synth.stream_key(seed, "q_logits"), 0, V)
+    p = np.exp(zp - zp.max()); p = (p / p.sum()).astype(np.float32)
+    q = np.exp(zq - zq.max()); q = (q / q.sum()).astype(np.float32)
+    x = synth.sample_rows_np(np.broadcast_to(q, (n, V)), synth.u53_np(synth.stream_key(seed, "u_draft"), 0, n))
+    ua = synth.u24_np(synth.stream_key(seed, "u_accept"), 0, n).reshape(n, 1)
+    ur = synth.u24_np(synth.stream_key(seed, "u_resample"), 0, n)
+    P = torch.from_numpy(p).to(DEV).expand(n, 1, V).contiguous()
+    Q = torch.from_numpy(q).to(DEV).expand(n, 1, V).contiguous()
+    acc, nxt = mm.block_accept_rejection(P, Q, torch.from_numpy(x.reshape(n, 1)).to(DEV),
+                                         torch.from_numpy(ua).to(DEV), torch.from_numpy(ur).to(DEV))
+    acc, nxt = acc.cpu().numpy(), nxt.cpu().numpy()
+    emitted = np.where(acc == 1, x, nxt)
+    counts = np.bincount(emitted, minlength=V)
+    expect = p.astype(np.float64) / p.astype(np.float64).sum() * n
+    chi2 = float(((counts - expect) ** 2 / expect).sum())
+    assert chi2 <= 37.697, chi2
+
+
+# ---------------------------------------------------------- stacked layers --
+
+def test_multilayer_each_layer():
+    """Every layer of the 8-layer stack at full size, fed its own seeded
+    input: RMSNorm -> route -> permute -> FFN -> combine with residual."""
+    sh = synth.SHAPES["multilayer"]
+    for layer in range(sh.layers):
+        L = Layer(sh, layer, DEV)
+        xn = mm.moe_rms_norm(L.x)
+        idx, w, off, sp, pr = _route_permute(L, sh)
+        y, ws = mm.mxfp4_moe_ffn(xn, sh.k, *L.w, off, sp)
+        out = mm.moe_combine(y, pr, w, residual=L.x)
+        xn_ref = omoe.rms_norm(L.x_f64())
+        assert_ffn_close(bf16_to_f64(xn), xn_ref, f"layer {layer} rms_norm")
+        roff = off.cpu().numpy()
+        rsp = sp.cpu().numpy()
+        ridx, rw, _ = omoe.route_topk(L.logits_np, sh.k)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        e = _sample_experts(omoe.permute(ridx, sh.E)[0], 1)[0]
+        r0, r1 = int(roff[e]), int(roff[e + 1])
+        _, ye = omoe.expert_ffn(xn_ref[rsp[r0:r1] // sh.k], *L.oracle_weights(e), sh.I)
+        assert_ffn_close(y.cpu().numpy()[r0:r1], ye, f"layer {layer} expert {e}")
+        del L
+
+
+def test_multilayer_chain_within_stack_gain():
+    """The whole 8-layer stack for a sampled token (tokens are independent in
+    MoE layers whose router logits are given), from seeded inputs only.
+
+    The stack is ill-conditioned: each SwiGLU layer is quadratic in its input
+    and lifts activations by ~1e8, so a relative difference at one layer grows
+    layer by layer.  The oracle measures that growth itself -- it reruns the
+    stack with layer 0's expert output perturbed by 1e-4 (random signs) and
+    takes kappa = final deviation / layer-0 deviation.  The GPU must match at
+    layer 0 within the FFN tolerance, and at the last layer within
+    max(2e-3, 4 * kappa * its layer-0 error)."""
+    sh = synth.SHAPES["multilayer"]
+    t = 97
+    L0 = Layer(sh, 0, DEV, with_weights=False)
+    resid = L0.x.clone()
+    ws = None
+    gpu_layers = []
+    for layer in range(sh.layers):
+        L = Layer(sh, layer, DEV)
+        xn = mm.moe_rms_norm(resid)
+        idx, w, off, sp, pr = _route_permute(L, sh)
+        y, ws = mm.mxfp4_moe_ffn(xn, sh.k, *L.w, off, sp, workspace=ws)
+        resid = mm.moe_combine(y, pr, w, residual=resid)
+        gpu_layers.append(bf16_to_f64(resid[t:t + 1]))
+        del L
+    rng = np.random.default_rng(1234)
+    sign = rng.choice([-1.0, 1.0], size=(sh.k, sh.H))
+    r = np.repeat(L0.x_f64()[t:t + 1], 2, axis=0)         # row 0 exact, row 1 perturbed
+    ref_layers, pert_layers = [], []
+    for layer in range(sh.layers):
+        lg = synth.router_logits(sh, layer)[t:t + 1]
+        xn = omoe.rms_norm(r)
+        ridx, rw, _ = omoe.route_topk(lg, sh.k)
+        ys = np.zeros((2, sh.k, sh.H))
+        for j in range(sh.k):
+            e = int(ridx[0, j])
+            wts = (synth.weight_codes_np(sh, "w13", e, layer), synth.weight_scales_np(sh, "w13", e, layer),
+                   synth.weight_codes_np(sh, "w2", e, layer), synth.weight_scales_np(sh, "w2", e, layer))
+            _, ys[:, j] = omoe.expert_ffn(xn, *wts, sh.I)
+        if layer == 0:
+            ys[1] *= 1.0 + 1e-4 * sign
+        nxt = np.zeros_like(r)
+        for c in range(2):
+            nxt[c], _ = omoe.combine(ys[c], np.arange(sh.k, dtype=np.int32), rw, r[c:c + 1])
+        r = nxt
+        ref_layers.append(r[0:1].copy())
+        pert_layers.append(r[1:2].copy())
+    from gpu_helpers import rel_l2
+    kappa = rel_l2(pert_layers[-1], ref_layers[-1]) / rel_l2(pert_layers[0], ref_layers[0])
+    e0 = rel_l2(gpu_layers[0], ref_layers[0])
+    eL = rel_l2(gpu_layers[-1], ref_layers[-1])
+    print(f"stack gain kappa={kappa:.1f}  gpu rel-L2 layer0={e0:.2e} layer{sh.layers - 1}={eL:.2e}")
+    print("per-layer gpu rel-L2:", [f"{rel_l2(g, r):.2e}" for g, r in zip(gpu_layers, ref_layers)])
+    print("per-layer perturbed rel-L2:", [f"{rel_l2(g, r):.2e}" for g, r in zip(pert_layers, ref_layers)])
+    assert e0 <= 2e-3
+    assert eL <= max(2e-3, 4 * kappa * e0), (kappa, e0, eL)
+
+
+# ------------------------------------------------------------ argument errors --
+
+def test_invalid_arguments_return_codes():
+    L = mm.lib()
+    assert L.moe_route_topk(None, 4, 8, 9, None, None, None) == 1       # k > E
+    assert L.moe_route_topk(None, 4, 2000, 2, None, None, None) == 2    # E > 1024
+    assert L.moe_permute(None, 4, 0, 8, None, None, None, None) == 1
+    assert L.mxfp4_moe_ffn_variant(None, 4, 200, 128, 8, 2, *([None] * 8), 0, 0, None) == 1
+    assert L.block_accept_greedy(None, None, 1, 33, 10, None, None, None) == 1
+    assert L.block_accept_rejection(None, None, None, None, None, 1, 4, (1 << 24) + 1,
+                                    None, None, None) == 1
+    # workspace too small
+    sh = synth.SHAPES["tiny"]
+    Ly = Layer(sh, 0, DEV)
+    idx, w, off, sp, pr = _route_permute(Ly, sh)
+    small = torch.empty(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(mm.MoeError) as ei:
+        mm.mxfp4_moe_ffn(Ly.x, sh.k, *Ly.w, off, sp, workspace=small)
+    assert ei.value.status == 4

@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--workload", default="batch1", choices=list(synth.SHAPES))
     ap.add_argument("--variant", type=int, default=0, help="FFN kernel: 0 auto, 1 FMA, 2 tensor")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the expert count (smaller cases for profiler captures)")
     return ap.parse_args()
 
 
@@ -279,6 +283,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     sh = synth.SHAPES[args.workload]
+    if args.experts:
+        sh = synth.Shape(**{**sh.__dict__, "E": args.experts, "name": f"{sh.name}-E{args.experts}"})
 
     if args.impl == "reference":
         if rank != 0:
@@ -330,20 +336,48 @@ def main():
         if world > 1:
             torch.distributed.barrier()
 
+    # CUDA graph of one step (launch gaps removed); eager launches otherwise
+    graph = None
+    if not args.no_graph:
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            wl.step(variant)
+        torch.cuda.current_stream().wait_stream(stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            wl.step(variant)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+
     clocks = ClockSampler(local)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record()
     for i in range(args.steps):
-        wl.step(variant, evs[i])
+        if graph is not None:
+            graph.replay()
+        else:
+            wl.step(variant)
     t_end.record()
     torch.cuda.synchronize()
     barrier()
-    clk = clocks.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
+    # per-call breakdown on eager launches, events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        wl.step(variant, evs[i])
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    eager_ms = e0.elapsed_time(e1) / args.steps
     ffn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     tail_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
@@ -352,7 +386,10 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
 
-    e2e_ms, h2d, d2h = e2e_time(wl, variant, args.steps, 3)
+    if args.no_e2e:
+        e2e_ms, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_ms, h2d, d2h = e2e_time(wl, variant, args.steps, 3)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -363,7 +400,8 @@ def main():
     vname = {0: "auto", 1: "fma", 2: "tensor"}[variant]
     traffic = load_traffic(sh.name, vname)
     tokens = sh.T * world
-    launches_per_step = 6 * (sh.layers if sh.layers > 1 else 1)
+    # route, permute, FFN (3 kernels), combine, greedy
+    launches_per_step = 7
     line = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -373,13 +411,14 @@ def main():
                                f"S={sh.S} x K={sh.K} block, greedy over V={sh.V}",
                    "global_batch_tokens": tokens, "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "inputs larger than L2: %.2f GB of expert weights read per step" % (act_bytes / 1e9),
-                   "ffn_variant": vname},
+                   "ffn_variant": vname, "timing": "CUDA graph replay" if graph is not None else "eager"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "mxfp4_moe_ffn (GEMM-1+SwiGLU and GEMM-2 launches)",
                      "algorithmic_bytes": act_bytes, "active_experts": n_act,
                      "peak_source": f"{peak_kind} hbm_gbs"},
-        "breakdown_ms": {"route+permute": route_ms, "ffn": ffn_ms, "combine+greedy": tail_ms},
+        "breakdown_ms": {"route+permute": route_ms, "ffn": ffn_ms, "combine+greedy": tail_ms,
+                         "eager_step": eager_ms, "graph_step": ms if graph is not None else None},
         "ffn_tflops": wl.ffn_flops() / (ffn_ms * 1e-3) / 1e12,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -119,8 +119,8 @@ int moe_permute(const int32_t *topk_idx, int T, int k, int E,
  *                  mxfp4_moe_ffn_workspace_bytes(T, k, H, I) bytes, 256-byte
  *                  aligned; its contents on entry do not matter.
  *   Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
- *   The kernel variant is chosen from the average number of rows per expert
- *   (see mxfp4_moe_ffn_variant).
+ *   The kernel variant: the tensor-core one wherever its limits allow
+ *   (H >= 512), else the FMA one (see mxfp4_moe_ffn_variant).
  */
 size_t mxfp4_moe_ffn_workspace_bytes(int T, int k, int H, int I);
 
@@ -133,7 +133,7 @@ int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
 
 /* Kernel variants of mxfp4_moe_ffn. */
 enum {
-  MOE_FFN_AUTO = 0,   /* pick by T*k / E                                  */
+  MOE_FFN_AUTO = 0,   /* tensor cores if H >= 512, else FMA               */
   MOE_FFN_FMA = 1,    /* dequantise to registers, float FMA (small N)     */
   MOE_FFN_TENSOR = 2  /* tcgen05 block-scaled MMA, TMEM accumulators      */
 };

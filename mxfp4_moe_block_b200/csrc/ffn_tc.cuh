@@ -591,10 +591,13 @@ inline size_t tc_workspace_bytes(size_t P, int H, int I) {
          align256_tc(2 * P * I / 32);
 }
 
-// Tensor cores pay off once an expert sees several tokens on average.
-inline bool tc_prefer(size_t P, int E) {
-  const size_t used = P < (size_t)E ? P : (size_t)E;
-  return used > 0 && P >= 4 * used;
+// The tensor-core variant streams the weights with TMA and needs no
+// dequantisation, so it is the default wherever its shape limits allow
+// (scale rows of at least 16 bytes: H >= 512).
+inline bool tc_prefer(size_t P, int E, int H) {
+  (void)P;
+  (void)E;
+  return H >= 512;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,

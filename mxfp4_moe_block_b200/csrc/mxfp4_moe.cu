@@ -161,7 +161,7 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
   const DeviceInfo *dev = device_info();
   if (!dev) return MOE_ERR_CUDA;
   const size_t P = (size_t)T * k;
-  if (variant == MOE_FFN_AUTO) variant = tc_prefer(P, E) ? MOE_FFN_TENSOR : MOE_FFN_FMA;
+  if (variant == MOE_FFN_AUTO) variant = tc_prefer(P, E, H) ? MOE_FFN_TENSOR : MOE_FFN_FMA;
 
   const WsLayout wl = ws_layout(T, k, H, I);
   uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);

@@ -152,6 +152,37 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
 const uint16_t *mxfp4_moe_ffn_workspace_h(const void *workspace);
 
 /*
+ * mxfp4_moe_ffn_noalloc -- mxfp4_moe_ffn for callers that cannot allocate.
+ *   The pages have no counterpart to this call; it exists for users of the
+ *   library that are not allowed to allocate device memory: plugins hosted by
+ *   an engine that reserves all device memory up front and hands its plugins
+ *   no allocator, and latency-critical loops in which a cudaMalloc/cudaFree
+ *   (cudaFree synchronises the device) is not acceptable.  Same contract as
+ *   mxfp4_moe_ffn, except that the scratch space comes from an array of
+ *   MOE_NOALLOC_SCRATCH_BYTES in the library's own device global memory,
+ *   which every GPU that loads the library holds until the process exits.
+ *   The caller still passes inputs and outputs.
+ *   - Problems whose scratch need (mxfp4_moe_ffn_workspace_bytes) exceeds
+ *     MOE_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE before
+ *     anything is launched.  8 MiB covers T*k <= 64 pairs at H = 7168,
+ *     I = 2048 (one 8-token block with top-8 routing).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents (the FFN writes every scratch byte it reads, so nothing needs
+ *     clearing).  Calls whose executions overlap on the GPU -- on different
+ *     streams, or from different host threads -- race on it; serialise them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
+                          const uint8_t *w13_codes, const uint8_t *w13_scales,
+                          const uint8_t *w2_codes, const uint8_t *w2_scales,
+                          const int32_t *expert_offsets, const int32_t *sorted_pair,
+                          float *y, moe_stream_t stream);
+
+/*
  * moe_combine -- weighted sum of each token's k expert outputs.
  *   out[t] = bf16( sum_{j<k} topk_w[t,j] * y[pair_row[t*k+j]] + residual[t] )
  *   in float, slots summed in order j = 0..k-1, residual added last.

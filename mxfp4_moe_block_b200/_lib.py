@@ -35,6 +35,8 @@ SIGNATURES = {
                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_size,
                                        _c_int, _vp]),
     "mxfp4_moe_ffn_workspace_h": (_vp, [_vp]),
+    "mxfp4_moe_ffn_noalloc": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                       _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_combine": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "moe_rms_norm": (_c_int, [_vp, _c_int, _c_int, _c_float, _vp, _vp]),
     "block_accept_greedy": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
@@ -148,6 +150,29 @@ def mxfp4_moe_ffn(x, k, w13_codes, w13_scales, w2_codes, w2_scales, expert_offse
         _ptr(y, torch.float32, "y"), _ptr(workspace), workspace.numel(), variant,
         _stream(stream)), "mxfp4_moe_ffn")
     return y, workspace
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def mxfp4_moe_ffn_noalloc(x, k, w13_codes, w13_scales, w2_codes, w2_scales, expert_offsets,
+                          sorted_pair, y=None, stream=None):
+    """mxfp4_moe_ffn without a caller-supplied workspace: the library uses its
+    own fixed device scratch (NOALLOC_SCRATCH_BYTES), so the call allocates
+    nothing when ``y`` is given.  For callers that may not allocate device
+    memory; calls that overlap on the GPU share that scratch and race."""
+    T, H = x.shape
+    E, twoI, _ = w13_codes.shape
+    I = twoI // 2
+    if y is None:
+        y = torch.empty((T * k, H), dtype=torch.float32, device=x.device)
+    _check(lib().mxfp4_moe_ffn_noalloc(
+        _ptr(x, torch.bfloat16, "x"), T, H, I, E, k,
+        _ptr(w13_codes, torch.uint8, "w13_codes"), _ptr(w13_scales, torch.uint8, "w13_scales"),
+        _ptr(w2_codes, torch.uint8, "w2_codes"), _ptr(w2_scales, torch.uint8, "w2_scales"),
+        _ptr(expert_offsets, torch.int32), _ptr(sorted_pair, torch.int32),
+        _ptr(y, torch.float32, "y"), _stream(stream)), "mxfp4_moe_ffn_noalloc")
+    return y
 
 
 def workspace_h(workspace, P, I):

@@ -192,6 +192,53 @@ int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
                                MOE_FFN_AUTO, stream);
 }
 
+// -------------------------------------------------------- FFN, no alloc --
+// Scratch of mxfp4_moe_ffn_noalloc: a fixed array in the library's own
+// device global memory, shared by every call on a device.  Host code must
+// not hand the symbol itself to a kernel (on the host it names a host-side
+// stand-in); its device address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+}  // namespace
+
+int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
+                          const uint8_t *w13_codes, const uint8_t *w13_scales,
+                          const uint8_t *w2_codes, const uint8_t *w2_scales,
+                          const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
+                          moe_stream_t stream) {
+  if (T < 0 || k < 1 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  if (mxfp4_moe_ffn_workspace_bytes(T, k, H, I) > (size_t)MOE_NOALLOC_SCRATCH_BYTES) {
+    fprintf(stderr,
+            "mxfp4_moe_ffn_noalloc: T=%d k=%d H=%d I=%d needs %zu scratch bytes, more than the "
+            "built-in %u\n",
+            T, k, H, I, mxfp4_moe_ffn_workspace_bytes(T, k, H, I),
+            (unsigned)MOE_NOALLOC_SCRATCH_BYTES);
+    return MOE_ERR_WORKSPACE;
+  }
+  int dev;
+  const int st = current_device(&dev);
+  if (st != MOE_OK) return st;
+  void *scratch;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+      }
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return mxfp4_moe_ffn_variant(x, T, H, I, E, k, w13_codes, w13_scales, w2_codes, w2_scales,
+                               expert_offsets, sorted_pair, y, scratch,
+                               (size_t)MOE_NOALLOC_SCRATCH_BYTES, MOE_FFN_AUTO, stream);
+}
+
 // ---------------------------------------------------------------- combine --
 int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w, int T, int k,
                 int H, const uint16_t *residual, uint16_t *out, moe_stream_t stream) {

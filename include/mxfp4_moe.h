@@ -133,9 +133,14 @@ int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
 
 /* Kernel variants of mxfp4_moe_ffn. */
 enum {
-  MOE_FFN_AUTO = 0,   /* tensor cores if H >= 512, else FMA               */
-  MOE_FFN_FMA = 1,    /* dequantise to registers, float FMA (small N)     */
-  MOE_FFN_TENSOR = 2  /* tcgen05 block-scaled MMA, TMEM accumulators      */
+  MOE_FFN_AUTO = 0,      /* tensor cores if H >= 512, else FMA                   */
+  MOE_FFN_FMA = 1,       /* dequantise to registers, float FMA                   */
+  MOE_FFN_TENSOR = 2,    /* tcgen05 block-scaled MMA: TENSOR_F4 if H, I are
+                            multiples of 256, else TENSOR_F8                      */
+  MOE_FFN_TENSOR_F8 = 3, /* kind::mxf8f6f4: padded E2M1 weights x two E4M3
+                            activation terms                                      */
+  MOE_FFN_TENSOR_F4 = 4  /* kind::mxf4: packed E2M1 weights x four E2M1
+                            activation terms (H, I multiples of 256)              */
 };
 
 /* Same contract as mxfp4_moe_ffn with an explicit kernel variant. */

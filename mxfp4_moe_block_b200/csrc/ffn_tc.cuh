@@ -137,10 +137,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 }
 constexpr uint32_t kSwizzle128B = 2, kSwizzleNone = 0;
 
-// Instruction descriptor of mxf8f6f4.block_scale: A = E2M1, B = E4M3,
-// E8M0 scales, M = 128, K-major A and B.
-__device__ __forceinline__ uint32_t idesc_mxf8f6f4(int n, uint32_t sf_id) {
-  return (sf_id << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
+// Instruction descriptor of a block-scaled MMA with E8M0 scales, M = 128,
+// K-major A and B: a/b formats (mxf8f6f4: 5 = E2M1, 0 = E4M3; mxf4: 1 =
+// E2M1), N, and the byte of the scale word each operand's scales start at.
+__device__ __forceinline__ uint32_t idesc_block_scaled(uint32_t afmt, uint32_t bfmt, int n,
+                                                       uint32_t sf_id) {
+  return (sf_id << 4) | (afmt << 7) | (bfmt << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
          ((128u >> 4) << 24) | (sf_id << 29);
 }
 
@@ -151,6 +153,17 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, u
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %6, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate));
 }
@@ -187,17 +200,35 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// --------------------------------------------- two-term E4M3 block encoding --
+// ------------------------------------------------ activation block encodings --
+//
+// The tensor cores take the activations (bf16 x, and GEMM-1's bf16 output h)
+// as a short sum of narrow terms, each with its own E8M0 scale per 32
+// elements: v = sum_t 2^(s_t) * c_t.  Term t encodes what terms 0..t-1 left
+// over.  Two E4M3 terms (kind::mxf8f6f4) or four E2M1 terms (kind::mxf4)
+// leave less than ~2^-18 (E4M3) / ~2^-16 (E2M1) of the block's largest
+// element; the error of the dot products is below 1e-4 relative, far under
+// the FFN tolerance.  Both encoders are warp-cooperative: lane l holds
+// element l of one 32-element block.
 
-// Exponent s of a block scale 2^s for block maximum amax (> 0): amax / 2^s
-// lies in [128, 256), inside E4M3's range (max 448).
-__device__ __forceinline__ int block_exp(float amax) {
+
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(127 + s) << 23); }
+
+// E4M3 term: scale exponent with amax / 2^s in [128, 256) (E4M3 max 448).
+__device__ __forceinline__ int e4m3_block_exp(float amax) {
   const int be = (int)((__float_as_uint(amax) >> 23) & 0xff);
   const int e = (be == 0 ? -126 : be - 127) - 7;
   return max(-126, min(126, e));
 }
 
-__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(127 + s) << 23); }
+// E2M1 term: scale exponent with amax / 2^s in (3, 6] (E2M1 max 6).
+__device__ __forceinline__ int e2m1_block_exp(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int be = (int)((b >> 23) & 0xff);
+  int e = (be == 0 ? -126 : be - 127) - 2;
+  if ((b & 0x7fffffu) > 0x400000u) e += 1;     // mantissa above 1.5: use 2^(e+1)
+  return max(-126, min(125, e));
+}
 
 __device__ __forceinline__ uint8_t to_e4m3(float v) {
   return (uint8_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
@@ -206,36 +237,91 @@ __device__ __forceinline__ float from_e4m3(uint8_t q) {
   __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q, __NV_E4M3);
   return __half2float(*reinterpret_cast<__half *>(&h));
 }
-
-// Warp-cooperative: lane l holds element l of one 32-element block.
-// Produces the two E4M3 codes of the lane and the two scale bytes.
-__device__ __forceinline__ void split2(float v, uint8_t &q1, uint8_t &q2, uint8_t &sb1,
-                                       uint8_t &sb2) {
-  const float a1 = warp_max(fabsf(v));
-  int s1 = 0;
-  float r = v;
-  if (a1 > 0.f) {
-    s1 = block_exp(a1);
-    q1 = to_e4m3(v * pow2f(-s1));
-    r = v - from_e4m3(q1) * pow2f(s1);
-  } else {
-    q1 = 0;
-  }
-  const float a2 = warp_max(fabsf(r));
-  int s2 = 0;
-  if (a2 > 0.f) {
-    s2 = block_exp(a2);
-    q2 = to_e4m3(r * pow2f(-s2));
-  } else {
-    q2 = 0;
-  }
-  sb1 = (uint8_t)(127 + s1);
-  sb2 = (uint8_t)(127 + s2);
+__device__ __forceinline__ uint32_t to_e2m1(float v) {
+  return (uint32_t)__nv_cvt_float_to_fp4(v, __NV_E2M1, cudaRoundNearest) & 0xfu;
 }
 
-// Activation operand of GEMM-1: for every sorted row r (token sp[r]/k), the
-// two E4M3 terms of x[token] as B rows 2r and 2r+1, [2P, H], and their scale
-// bytes [2P, H/32].  One warp per 32-element block.
+// Two E4M3 terms: codes q[0..1] of this lane, scale bytes sb[0..1] (warp-uniform).
+__device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t (&sb)[2]) {
+  float r = v;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const float amax = warp_max(fabsf(r));
+    int s = 0;
+    uint32_t c = 0;
+    if (amax > 0.f) {
+      s = e4m3_block_exp(amax);
+      c = to_e4m3(r * pow2f(-s));
+      r -= from_e4m3((uint8_t)c) * pow2f(s);
+    }
+    q[t] = c;
+    sb[t] = (uint8_t)(127 + s);
+  }
+}
+
+// Four E2M1 terms: 4-bit codes q[0..3] of this lane, scale bytes sb[0..3].
+__device__ __forceinline__ void encode_e2m1x4(float v, uint32_t (&q)[4], uint8_t (&sb)[4]) {
+  float r = v;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const float amax = warp_max(fabsf(r));
+    int s = 0;
+    uint32_t c = 0;
+    if (amax > 0.f) {
+      s = e2m1_block_exp(amax);
+      c = to_e2m1(r * pow2f(-s));
+      r -= e2m1x2_to_f32x2(c).x * pow2f(s);
+    }
+    q[t] = c;
+    sb[t] = (uint8_t)(127 + s);
+  }
+}
+
+// Kind of tensor-core MMA used by the FFN.
+enum TcKind { KIND_F8 = 0, KIND_F4 = 1 };
+
+template <int KIND>
+struct TcKindCfg {
+  static constexpr int kTerms = KIND == KIND_F4 ? 4 : 2;        // B rows per token
+  static constexpr int kStageK = KIND == KIND_F4 ? 256 : 128;   // K elements per stage
+  static constexpr int kKGroups = kStageK / 128;                // 4-scale groups per stage
+  static constexpr int kMmaK = kStageK / 4;                     // 4 MMAs per stage
+  static constexpr uint32_t kABytes = 128u * kStageK / 2;       // packed weight bytes per stage
+  static constexpr int kBRowBytesPerK2 = KIND == KIND_F4 ? 1 : 2;  // B row bytes = K * this / 2
+};
+
+// Stores one lane's encoded element n of activation row r (terms in rows
+// T*r + t) and the block's scale bytes.
+template <int KIND>
+__device__ __forceinline__ void store_terms(float v, size_t r, int n, int kdim, uint8_t *q_out,
+                                            uint8_t *s_out, int lane, bool valid) {
+  if (KIND == KIND_F4) {
+    uint32_t q[4];
+    uint8_t sb[4];
+    encode_e2m1x4(v, q, sb);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t hi = __shfl_down_sync(FULL, q[t], 1);
+      if (valid && !(lane & 1))
+        q_out[(4 * r + t) * (size_t)(kdim / 2) + n / 2] = (uint8_t)(q[t] | (hi << 4));
+      if (valid && lane == 0) s_out[(4 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
+    }
+  } else {
+    uint32_t q[2];
+    uint8_t sb[2];
+    encode_e4m3x2(v, q, sb);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (valid) q_out[(2 * r + t) * (size_t)kdim + n] = (uint8_t)q[t];
+      if (valid && lane == 0) s_out[(2 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
+    }
+  }
+}
+
+// Activation operand of GEMM-1: for every sorted row r (token sp[r]/k) the
+// terms of x[token] as B rows T*r + t, and their scale bytes.  One warp per
+// 32-element block.
+template <int KIND>
 __global__ void __launch_bounds__(256)
 split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, int P, int k,
                int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
@@ -247,75 +333,79 @@ split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, i
     const int r = (int)(w / nb), b = (int)(w % nb);
     const int t = __ldg(sp + r) / k;
     const float v = __uint_as_float((uint32_t)__ldg(x + (size_t)t * H + b * 32 + lane) << 16);
-    uint8_t q1, q2, s1, s2;
-    split2(v, q1, q2, s1, s2);
-    xq[(size_t)(2 * r) * H + b * 32 + lane] = q1;
-    xq[(size_t)(2 * r + 1) * H + b * 32 + lane] = q2;
-    if (lane == 0) {
-      xs[(size_t)(2 * r) * nb + b] = s1;
-      xs[(size_t)(2 * r + 1) * nb + b] = s2;
-    }
+    store_terms<KIND>(v, (size_t)r, b * 32 + lane, H, xq, xs, lane, true);
   }
 }
 
 // ------------------------------------------------------------- the kernel --
 
 struct TcMaps {
-  CUtensorMap a;        // weights: [E*rows, K] E2M1 (16U4_ALIGN16B), box 128 x 64 rows
-  CUtensorMap b[5];     // activations: [2P, K] E4M3, box 128 x {16,32,64,128,256} rows
+  CUtensorMap a;        // weights [E*rows, K]: box 128 (padded E2M1) or 128 B (packed) x 64 rows
+  CUtensorMap b[5];     // activation terms [T*P, row bytes]: box 128 B x {16,...,256} rows
 };
 
 struct TcArgs {
   const uint8_t *a_scales;   // [E*rows, K/32]
-  const uint8_t *b_scales;   // [2P, K/32]
+  const uint8_t *b_scales;   // [T*P, K/32]
   const int32_t *off;        // [E+1]
   int E, K, rows_per_expert, P;
-  int I;                     // GEMM-1: the gate/up split; GEMM-2: unused
+  int I;                     // GEMM-1: the gate/up split
   int H;                     // y row length (GEMM-2)
-  int b_box[5];              // rows of each B box (clamped to 2P)
+  int b_box[5];              // rows of each B box (clamped to T*P)
   // GEMM-1 outputs
   uint16_t *h;               // [P, I] bf16
-  uint8_t *hq;               // [2P, I] E4M3 terms
-  uint8_t *hs;               // [2P, I/32] scale bytes
+  uint8_t *hq;               // activation terms of h
+  uint8_t *hs;               // their scale bytes
   // GEMM-2 output
   float *y;                  // [P, H]
 };
 
-template <int BN>
+template <int KIND, int BN>
 struct TcCfg {
-  static constexpr int kStages = BN <= 32 ? 10 : BN <= 64 ? 8 : BN <= 128 ? 6 : 4;
-  static constexpr int kSfbChunks = (BN + 127) / 128;
-  static constexpr int kA = 128 * 128;                 // bytes of one A stage
+  using Kd = TcKindCfg<KIND>;
+  static constexpr int kRowChunks = (BN + 127) / 128;               // 128-row scale chunks of B
+  static constexpr int kA = 128 * 128;                              // smem bytes of one A stage
   static constexpr int kB = BN * 128;
-  static constexpr int kSfa = 512;
-  static constexpr int kSfb = 512 * kSfbChunks;
-  static constexpr int kSfCols = 4 + 4 * kSfbChunks;   // TMEM columns per stage
-  static constexpr int kAcc = BN <= 128 ? 2 : 1;        // accumulator buffers
-  static constexpr int kUsed = kAcc * BN + kStages * kSfCols;
+  static constexpr int kSfa = 512 * Kd::kKGroups;
+  static constexpr int kSfb = 512 * Kd::kKGroups * kRowChunks;
+  static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
+  static constexpr int kFixed = 1024 + 2048 + 2 * 1025 * 4 + 1024;  // barriers, xchg, table, slack
+  static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
+  static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
+  static constexpr int kSfCols = 4 * Kd::kKGroups * (1 + kRowChunks);   // TMEM columns per stage
+  static constexpr int kAcc = BN <= 128 ? 2 : 1;                   // accumulator buffers
+  // Independent accumulation chains per buffer: with few B columns each MMA
+  // is tiny and a single chain would run at MMA latency; MMA kk of a stage
+  // accumulates into chain kk % kChains and the epilogue adds the chains.
+  static constexpr int kChains = BN <= 32 ? 4 : BN <= 64 ? 2 : 1;
+  static constexpr int kAccCols = kAcc * kChains * BN;
+  static constexpr int kUsed = kAccCols + kStages * kSfCols;
   static constexpr int kTmemCols = kUsed <= 128 ? 128 : kUsed <= 256 ? 256 : 512;
   static_assert(kUsed <= 512, "TMEM budget");
   static constexpr int kOffB = kStages * kA;
   static constexpr int kOffSfa = kOffB + kStages * kB;
   static constexpr int kOffSfb = kOffSfa + kStages * kSfa;
   static constexpr int kOffBar = kOffSfb + kStages * kSfb;
-  static constexpr int kOffXchg = kOffBar + 1024;                // 64 x 8 floats
+  static constexpr int kOffXchg = kOffBar + 1024;                // 64 rows x 4 tokens (float)
   static constexpr int kOffTab = kOffXchg + 2048;                 // active list + prefix
-  static constexpr int kSmem = kOffTab + 2 * 1025 * 4 + 1024;     // + 1 KB alignment slack
+  static constexpr int kSmem = kOffTab + 2 * 1025 * 4 + 1024;     // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
 constexpr int TC_THREADS = 256;
 
-template <int MODE, int BN>
+template <int KIND, int MODE, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<KIND, BN>;
+  using Kd = TcKindCfg<KIND>;
+  constexpr int T = Kd::kTerms;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *empty = full + C::kStages;
-  uint64_t *acc_full = empty + C::kStages;     // [kAcc]
-  uint64_t *acc_empty = acc_full + 2;          // [kAcc]
+  uint64_t *acc_full = empty + C::kStages;     // [2]
+  uint64_t *acc_empty = acc_full + 2;          // [2]
   volatile int *abort = reinterpret_cast<volatile int *>(acc_empty + 2);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 3);
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
@@ -324,7 +414,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mtiles = MODE == 1 ? a.I / 64 : a.rows_per_expert / 128;
-  const int ksteps = a.K / 128;
+  const int ksteps = a.K / Kd::kStageK;
 
   // tile table: active experts and the prefix of their tile counts
   if (warp == 0) {
@@ -332,9 +422,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
       const int cnt = e < a.E ? __ldg(a.off + e + 1) - __ldg(a.off + e) : 0;
-      const int nt = cnt > 0 ? (2 * cnt + BN - 1) / BN : 0;
+      const int nt = cnt > 0 ? (T * cnt + BN - 1) / BN : 0;
       const unsigned b = __ballot_sync(FULL, nt > 0);
-      // inclusive scan of tiles among lanes
       int sc = nt * mtiles;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -378,21 +467,21 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   const int n_tiles = s_pre[n_act];
 
   // tile index -> (expert, m-block, first B row, B rows in the tile)
-  auto decode = [&](int t, int &e, int &mt, int &rowB, int &nB, int &r0, int &ne) {
+  auto decode = [&](int t, int &e, int &mt, int &rowB, int &nB) {
     int lo = 0, hi = n_act - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_pre[mid] <= t) lo = mid; else hi = mid - 1;
     }
     e = s_act[lo];
-    r0 = __ldg(a.off + e);
-    ne = __ldg(a.off + e + 1) - r0;
-    const int nt_cnt = (2 * ne + BN - 1) / BN;
+    const int r0 = __ldg(a.off + e);
+    const int ne = __ldg(a.off + e + 1) - r0;
+    const int nt_cnt = (T * ne + BN - 1) / BN;
     const int local = t - s_pre[lo];
     mt = local / nt_cnt;
     const int nt = local % nt_cnt;
-    rowB = 2 * r0 + nt * BN;
-    nB = min(BN, 2 * ne - nt * BN);
+    rowB = T * r0 + nt * BN;
+    nB = min(BN, T * ne - nt * BN);
   };
 
   if (warp == 0) {
@@ -403,16 +492,18 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       uint32_t phase = 0;
       int issued = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
-        int e, mt, rowB, nB, r0, ne;
-        decode(t, e, mt, rowB, nB, r0, ne);
+        int e, mt, rowB, nB;
+        decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
         const int bsel = ncol <= 16 ? 0 : ncol <= 32 ? 1 : ncol <= 64 ? 2 : ncol <= 128 ? 3 : 4;
         const uint32_t bbytes = (uint32_t)a.b_box[bsel] * 128u;
         const int arow = e * a.rows_per_expert + (MODE == 1 ? mt * 64 : mt * 128);
         for (int kt = 0; kt < ksteps; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
-          mbar_expect_tx(&full[stage], 128 * 128 / 2 + bbytes);
+          mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
           uint8_t *sa = smem + stage * C::kA;
+          // the box's inner coordinate is in elements (padded E2M1) or bytes
+          // (packed E2M1); both are kt * 128
           // rows 0-63 of the tile, then rows 64-127 (GEMM-1: gate, then up)
           tma_load_2d(sa, &maps.a, kt * 128, arow, &full[stage], pol_w);
           tma_load_2d(sa + 64 * 128, &maps.a, kt * 128, arow + (MODE == 1 ? a.I : 64),
@@ -434,31 +525,38 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
   } else if (warp == 1) {
     // --------------------------------------------------- scale loader --
+    // Per stage and 4-scale group g: scale bytes of the 128 A rows (and of
+    // the B rows) go straight into the 32 x 16-byte layout of tcgen05.cp:
+    // byte 16*(row%32) + 4*(row/32) + (k-block within the group).
     const uint32_t kb = a.K / 32;            // scale bytes per row
     int stage = 0;
     uint32_t phase = 0;
     for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
-      int e, mt, rowB, nB, r0, ne;
-      decode(t, e, mt, rowB, nB, r0, ne);
+      int e, mt, rowB, nB;
+      decode(t, e, mt, rowB, nB);
       const int ebase = e * a.rows_per_expert;
       for (int kt = 0; kt < ksteps; ++kt) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
         uint8_t *sfa = smem + C::kOffSfa + stage * C::kSfa;
         uint8_t *sfb = smem + C::kOffSfb + stage * C::kSfb;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {       // A rows lane + 32g
-          const int i = lane + 32 * g;
-          int row;
-          if (MODE == 1) row = ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64);
-          else row = ebase + mt * 128 + i;
-          cp_async4(sfa + 16 * lane + 4 * g, a.a_scales + (size_t)row * kb + kt * 4);
-        }
+        for (int g = 0; g < Kd::kKGroups; ++g) {
+          const uint32_t koff = (uint32_t)(kt * Kd::kKGroups + g) * 4;
 #pragma unroll
-        for (int g = 0; g < 4 * C::kSfbChunks; ++g) {
-          const int i = lane + 32 * g;
-          if (i < nB)
-            cp_async4(sfb + 512 * (g >> 2) + 16 * lane + 4 * (g & 3),
-                      a.b_scales + (size_t)(rowB + i) * kb + kt * 4);
+          for (int q = 0; q < 4; ++q) {       // A rows lane + 32q
+            const int i = lane + 32 * q;
+            int row;
+            if (MODE == 1) row = ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64);
+            else row = ebase + mt * 128 + i;
+            cp_async4(sfa + 512 * g + 16 * lane + 4 * q, a.a_scales + (size_t)row * kb + koff);
+          }
+#pragma unroll
+          for (int q = 0; q < 4 * C::kRowChunks; ++q) {
+            const int i = lane + 32 * q;
+            if (i < nB)
+              cp_async4(sfb + 512 * (g * C::kRowChunks + (q >> 2)) + 16 * lane + 4 * (q & 3),
+                        a.b_scales + (size_t)(rowB + i) * kb + koff);
+          }
         }
         cp_async_arrive_noinc(&full[stage]);
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -470,38 +568,56 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t sf_col0 = (uint32_t)(C::kAcc * BN);
+      const uint32_t sf_col0 = (uint32_t)C::kAccCols;
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
-        int e, mt, rowB, nB, r0, ne;
-        decode(t, e, mt, rowB, nB, r0, ne);
+        int e, mt, rowB, nB;
+        decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
         const int buf = it % C::kAcc;
         const uint32_t use = (uint32_t)(it / C::kAcc);
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort)) break;
         tc_fence_after();
-        const uint32_t acc_t = tmem + (uint32_t)(buf * BN);
+        const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
         bool ok = true;
         for (int kt = 0; kt < ksteps; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
-          fence_proxy_async();
+          // The scale bytes arrive by cp.async and are tracked by the same
+          // mbarrier; as in CUTLASS's cp.async-fed UMMA pipelines, the barrier
+          // wait is the only ordering tcgen05.cp needs.
           tc_fence_after();
+          // TMEM: per stage, the A scale groups then, per group, the B row chunks
           const uint32_t sfa_t = tmem + sf_col0 + stage * C::kSfCols;
-          const uint32_t sfb_t = sfa_t + 4;
+          const uint32_t sfb_t = sfa_t + 4 * Kd::kKGroups;
           const uint32_t sa = smem_u32(smem + C::kOffSfa + stage * C::kSfa);
           const uint32_t sb = smem_u32(smem + C::kOffSfb + stage * C::kSfb);
-          tc_cp_32x128b(sfa_t, smem_desc(sa, 0, 128, kSwizzleNone));
 #pragma unroll
-          for (int c = 0; c < C::kSfbChunks; ++c)
-            tc_cp_32x128b(sfb_t + 4 * c, smem_desc(sb + 512 * c, 0, 128, kSwizzleNone));
+          for (int g = 0; g < Kd::kKGroups; ++g) {
+            tc_cp_32x128b(sfa_t + 4 * g, smem_desc(sa + 512 * g, 0, 128, kSwizzleNone));
+#pragma unroll
+            for (int c = 0; c < C::kRowChunks; ++c)
+              tc_cp_32x128b(sfb_t + 4 * (g * C::kRowChunks + c),
+                            smem_desc(sb + 512 * (g * C::kRowChunks + c), 0, 128, kSwizzleNone));
+          }
           const uint32_t a_addr = smem_u32(smem + stage * C::kA);
           const uint32_t b_addr = smem_u32(smem + C::kOffB + stage * C::kB);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
+            // 32 bytes of each 128-byte row per MMA (K = 32 E4M3/E2M1-padded or 64 E2M1)
             const uint64_t ad = smem_desc(a_addr + 32 * kk, 16, 1024, kSwizzle128B);
             const uint64_t bd = smem_desc(b_addr + 32 * kk, 16, 1024, kSwizzle128B);
-            mma_mxf8f6f4(acc_t, ad, bd, idesc_mxf8f6f4(ncol, kk), sfa_t | ((uint32_t)kk << 30),
-                         sfb_t | ((uint32_t)kk << 30), (kt > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t acc = (kt > 0 || kk >= C::kChains) ? 1u : 0u;
+            const uint32_t d_t = acc_t + (uint32_t)((kk % C::kChains) * BN);
+            if (KIND == KIND_F4) {
+              const int g = kk >> 1;                     // scale group of this MMA
+              const uint32_t sfid = 2u * (kk & 1);      // two scale bytes per row
+              mma_mxf4(d_t, ad, bd, idesc_block_scaled(1, 1, ncol, sfid),
+                       (sfa_t + 4 * g) | (sfid << 30),
+                       (sfb_t + 4 * g * C::kRowChunks) | (sfid << 30), acc);
+            } else {
+              mma_mxf8f6f4(d_t, ad, bd, idesc_block_scaled(5, 0, ncol, kk),
+                           sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30), acc);
+            }
           }
           tc_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -512,57 +628,65 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------- epilogue --
+    // accumulator column T*j + t holds term t of token j of the tile
     const int q = warp - 4;                     // TMEM lane quarter
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    constexpr int kTokPerLd = 16 / T;           // tokens per 16-column load
     int it = 0;
     for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
-      int e, mt, rowB, nB, r0, ne;
-      decode(t, e, mt, rowB, nB, r0, ne);
+      int e, mt, rowB, nB;
+      decode(t, e, mt, rowB, nB);
       const int buf = it % C::kAcc;
       const uint32_t use = (uint32_t)(it / C::kAcc);
       if (!mbar_wait(&acc_full[buf], use & 1, abort)) break;
       tc_fence_after();
-      const uint32_t acc_t = tmem + (uint32_t)(buf * BN);
-      const int ntok = nB >> 1;                 // tokens in this tile (B rows come in pairs)
-      const int rtok0 = rowB >> 1;              // sorted row of the tile's first token
+      const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
+      const int ntok = nB / T;                  // tokens in this tile
+      const int rtok0 = rowB / T;               // sorted row of the tile's first token
       for (int c0 = 0; c0 < nB; c0 += 16) {
         float v[16];
         tc_ld16(acc_t + lane_base + (uint32_t)c0, v);
+#pragma unroll
+        for (int ch = 1; ch < C::kChains; ++ch) {
+          float w[16];
+          tc_ld16(acc_t + lane_base + (uint32_t)(ch * BN + c0), w);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += w[i];
+        }
+        float tok_sum[kTokPerLd];
+#pragma unroll
+        for (int j = 0; j < kTokPerLd; ++j) {
+          float sum = 0.f;
+#pragma unroll
+          for (int u = 0; u < T; ++u) sum += v[T * j + u];
+          tok_sum[j] = sum;
+        }
+        const int tok0 = c0 / T;
         if (MODE == 2) {
           const int m = mt * 128 + 32 * q + lane;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int tok = (c0 >> 1) + j;
-            if (tok < ntok) a.y[(size_t)(rtok0 + tok) * a.H + m] = v[2 * j] + v[2 * j + 1];
-          }
+          for (int j = 0; j < kTokPerLd; ++j)
+            if (tok0 + j < ntok) a.y[(size_t)(rtok0 + tok0 + j) * a.H + m] = tok_sum[j];
         } else {
           // rows 0-63 gate (quarters 0,1), 64-127 up (quarters 2,3)
           if (q >= 2) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) xchg[(32 * (q - 2) + lane) * 8 + j] = v[2 * j] + v[2 * j + 1];
+            for (int j = 0; j < kTokPerLd; ++j) xchg[(32 * (q - 2) + lane) * 8 + j] = tok_sum[j];
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
           if (q < 2) {
             const int n = mt * 64 + 32 * q + lane;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int tok = (c0 >> 1) + j;
-              const float g = v[2 * j] + v[2 * j + 1];
+            for (int j = 0; j < kTokPerLd; ++j) {
+              const int tok = tok0 + j;
+              const float g = tok_sum[j];
               const float u = xchg[(32 * q + lane) * 8 + j];
               const uint16_t hb = f32_to_bf16_bits(g / (1.f + expf(-g)) * u);
-              const float hv = __uint_as_float((uint32_t)hb << 16);
-              uint8_t q1, q2, s1, s2;
-              split2(hv, q1, q2, s1, s2);     // warp-uniform control flow
-              if (tok < ntok) {
-                const size_t r = (size_t)(rtok0 + tok);
-                a.h[r * a.I + n] = hb;
-                a.hq[(2 * r) * a.I + n] = q1;
-                a.hq[(2 * r + 1) * a.I + n] = q2;
-                if (lane == 0) {
-                  a.hs[(2 * r) * (a.I / 32) + n / 32] = s1;
-                  a.hs[(2 * r + 1) * (a.I / 32) + n / 32] = s2;
-                }
-              }
+              const bool valid = tok < ntok;
+              const size_t r = (size_t)(rtok0 + tok);
+              if (valid) a.h[r * a.I + n] = hb;
+              store_terms<KIND>(__uint_as_float((uint32_t)hb << 16), r, n, a.I, a.hq, a.hs,
+                                lane, valid);
             }
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -586,9 +710,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 
 inline size_t align256_tc(size_t n) { return (n + 255) & ~size_t(255); }
 
+// Operands of either kind: terms of x [T*P, H bytes*] and of h, plus scales
+// for up to 4 terms per row.
 inline size_t tc_workspace_bytes(size_t P, int H, int I) {
-  return align256_tc(2 * P * H) + align256_tc(2 * P * H / 32) + align256_tc(2 * P * I) +
-         align256_tc(2 * P * I / 32);
+  return align256_tc(2 * P * H) + align256_tc(4 * P * H / 32) + align256_tc(2 * P * I) +
+         align256_tc(4 * P * I / 32);
 }
 
 // The tensor-core variant streams the weights with TMA and needs no
@@ -621,42 +747,57 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // 2-D K-major tensor map: inner dimension `inner` elements, `rows` rows,
-// row pitch `pitch` bytes, box 128 x box_rows, 128-byte swizzle.
+// row pitch `pitch` bytes, box `box_inner` x `box_rows`, 128-byte swizzle.
 inline bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
-                     uint64_t rows, uint64_t pitch, uint32_t box_rows) {
+                     uint64_t rows, uint64_t pitch, uint32_t box_inner, uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {pitch};
-  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+// Weight map of one matrix [E*rows, K]: padded E2M1 (box 128 elements) for
+// kind::mxf8f6f4, packed bytes (box 128 bytes = 256 codes) for kind::mxf4.
+template <int KIND>
+inline bool make_weight_map(CUtensorMap *m, const uint8_t *codes, uint64_t K, uint64_t rows) {
+  if (KIND == KIND_F4)
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, rows, K / 2, 128, 64);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, codes, K, rows, K / 2, 128, 64);
+}
+
+template <int KIND, int BN>
 int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<KIND, BN>;
+  using Kd = TcKindCfg<KIND>;
+  constexpr int T = Kd::kTerms;
   const size_t P = (size_t)f.T * f.k;
   const int H = f.H, I = f.I, E = f.E;
+  const size_t xrow = (size_t)H * Kd::kBRowBytesPerK2 / 2;   // bytes per term row of x
+  const size_t hrow = (size_t)I * Kd::kBRowBytesPerK2 / 2;
   uint8_t *xq = ws;
   uint8_t *xs = xq + align256_tc(2 * P * H);
-  uint8_t *hq = xs + align256_tc(2 * P * H / 32);
+  uint8_t *hq = xs + align256_tc(4 * P * H / 32);
   uint8_t *hs = hq + align256_tc(2 * P * I);
 
-  static bool attr = false;
-  if (!attr) {
-    attr = true;
-    cudaFuncSetAttribute(tc_gemm_kernel<1, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static unsigned long long attr_done = 0;      // one bit per device
+  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
+    attr_done |= 1ull << dev;
+    cudaFuncSetAttribute(tc_gemm_kernel<KIND, 1, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          C::kSmem);
-    cudaFuncSetAttribute(tc_gemm_kernel<2, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(tc_gemm_kernel<KIND, 2, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          C::kSmem);
   }
   {
     const long blocks = (long)P * (H / 32);
     const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
-    split_x_kernel<<<grid, 256, 0, s>>>(f.x, f.sp, (int)P, f.k, H, xq, xs);
+    split_x_kernel<KIND><<<grid, 256, 0, s>>>(f.x, f.sp, (int)P, f.k, H, xq, xs);
   }
   TcMaps maps;
   TcArgs a{};
@@ -669,49 +810,59 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.hq = hq;
   a.hs = hs;
   a.y = f.y;
-  for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, 2 * P);
+  for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
 
-  // GEMM-1: W13 [E*2I, H] x x-terms [2P, H]
-  if (!make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, f.w13c, H, (uint64_t)E * 2 * I,
-                H / 2, 64))
-    return MOE_ERR_CUDA;
+  // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]
+  if (!make_weight_map<KIND>(&maps.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
   for (int i = 0; i < 5; ++i)
-    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, H, 2 * P, H, a.b_box[i]))
+    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
+                  a.b_box[i]))
       return MOE_ERR_CUDA;
   a.a_scales = f.w13s;
   a.b_scales = xs;
   a.K = H;
   a.rows_per_expert = 2 * I;
-  tc_gemm_kernel<1, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
+  tc_gemm_kernel<KIND, 1, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
-  // GEMM-2: W2 [E*H, I] x h-terms [2P, I]
-  if (!make_map(&maps.a, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, f.w2c, I, (uint64_t)E * H, I / 2,
-                64))
-    return MOE_ERR_CUDA;
+  // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
+  if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
   for (int i = 0; i < 5; ++i)
-    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, I, 2 * P, I, a.b_box[i]))
+    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
+                  a.b_box[i]))
       return MOE_ERR_CUDA;
   a.a_scales = f.w2s;
   a.b_scales = hs;
   a.K = I;
   a.rows_per_expert = H;
-  tc_gemm_kernel<2, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
+  tc_gemm_kernel<KIND, 2, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
-inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
-  if (f.H < 512 || f.I < 128) return MOE_ERR_UNSUPPORTED;   // scale rows of >= 16 bytes
+template <int KIND>
+inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   const size_t P = (size_t)f.T * f.k;
   const size_t used = P < (size_t)f.E ? P : (size_t)f.E;
-  const size_t rows = (2 * P + used - 1) / used;            // average B rows per expert
+  const size_t rows = (TcKindCfg<KIND>::kTerms * P + used - 1) / used;  // B rows per expert
   const size_t want = rows + rows / 2;
-  if (want <= 16) return tc_run<16>(f, ws, sms, s);
-  if (want <= 32) return tc_run<32>(f, ws, sms, s);
-  if (want <= 64) return tc_run<64>(f, ws, sms, s);
-  if (want <= 128) return tc_run<128>(f, ws, sms, s);
-  return tc_run<256>(f, ws, sms, s);
+  if (want <= 16) return tc_run<KIND, 16>(f, ws, sms, s);
+  if (want <= 32) return tc_run<KIND, 32>(f, ws, sms, s);
+  if (want <= 64) return tc_run<KIND, 64>(f, ws, sms, s);
+  if (want <= 128) return tc_run<KIND, 128>(f, ws, sms, s);
+  return tc_run<KIND, 256>(f, ws, sms, s);
+}
+
+// kind::mxf4 (packed FP4 weights, 4 activation terms) when K allows 256-wide
+// stages, else kind::mxf8f6f4.
+inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int kind) {
+  if (f.H < 512 || f.I < 128) return MOE_ERR_UNSUPPORTED;   // scale rows of >= 16 bytes
+  if (kind < 0) kind = (f.H % 256 == 0 && f.I % 256 == 0) ? KIND_F4 : KIND_F8;
+  if (kind == KIND_F4) {
+    if (f.H % 256 || f.I % 256) return MOE_ERR_UNSUPPORTED;
+    return tc_dispatch<KIND_F4>(f, ws, sms, s);
+  }
+  return tc_dispatch<KIND_F8>(f, ws, sms, s);
 }
 
 }  // namespace moe

@@ -150,7 +150,7 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
   if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
-  if (variant < MOE_FFN_AUTO || variant > MOE_FFN_TENSOR) return MOE_ERR_INVALID_ARG;
+  if (variant < MOE_FFN_AUTO || variant > MOE_FFN_TENSOR_F4) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !expert_offsets ||
       !sorted_pair || !y || !workspace)
@@ -169,7 +169,9 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
             expert_offsets, sorted_pair, reinterpret_cast<uint16_t *>(ws + wl.h), y,
             reinterpret_cast<float *>(ws + wl.x32), reinterpret_cast<float *>(ws + wl.h32)};
   cudaStream_t s = (cudaStream_t)stream;
-  if (variant == MOE_FFN_TENSOR) return tc_ffn(a, ws + wl.tc, dev->sms, s);
+  if (variant == MOE_FFN_TENSOR) return tc_ffn(a, ws + wl.tc, dev->sms, s, -1);
+  if (variant == MOE_FFN_TENSOR_F8) return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F8);
+  if (variant == MOE_FFN_TENSOR_F4) return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F4);
   const size_t n8 = (size_t)T * H / 8;
   x_to_f32_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8), 256, 0, s>>>(
       x, n8, a.x32);

@@ -140,8 +140,9 @@ def test_ffn_fma(name):
 
 
 @pytest.mark.parametrize("name", ["batch1", "serving", "dflash16", "multilayer"])
-def test_ffn_tensor(name):
-    _ffn_check(name, 0, mm.FFN_TENSOR)
+@pytest.mark.parametrize("variant", [3, 4], ids=["mxf8f6f4", "mxf4"])
+def test_ffn_tensor(name, variant):
+    _ffn_check(name, 0, variant)
 
 
 def test_ffn_tensor_small_shapes_and_bn_classes():
@@ -151,13 +152,15 @@ def test_ffn_tensor_small_shapes_and_bn_classes():
         sh = synth.Shape("tcs", H=512, I=256, E=E, k=k, S=1, K=K, V=64, seed=20 + K)
         L = Layer(sh, 0, DEV)
         idx, w, off, sp, pr = _route_permute(L, sh)
-        y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=mm.FFN_TENSOR)
         ridx, _, _ = omoe.route_topk(L.logits_np, sh.k)
         roff, rsp, _ = omoe.permute(ridx, sh.E)
         h_ref, y_ref = omoe.moe_ffn(L.x_f64(), sh.k, sh.I, L.oracle_weights, roff, rsp)
-        assert_ffn_close(bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I)), h_ref, f"h K={K}")
-        assert_ffn_close(y.cpu().numpy(), y_ref, f"y K={K}")
-        assert mm.moe_get_device_status() == (0, 0)
+        for variant in (mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4):
+            y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=variant)
+            assert_ffn_close(bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I)), h_ref,
+                             f"h K={K} variant {variant}")
+            assert_ffn_close(y.cpu().numpy(), y_ref, f"y K={K} variant {variant}")
+            assert mm.moe_get_device_status() == (0, 0)
 
 
 def test_ffn_one_expert_many_tokens():

@@ -203,13 +203,16 @@ __device__ __forceinline__ float warp_max(float v) {
 // ------------------------------------------------ activation block encodings --
 //
 // The tensor cores take the activations (bf16 x, and GEMM-1's bf16 output h)
-// as a short sum of narrow terms, each with its own E8M0 scale per 32
-// elements: v = sum_t 2^(s_t) * c_t.  Term t encodes what terms 0..t-1 left
-// over.  Two E4M3 terms (kind::mxf8f6f4) or four E2M1 terms (kind::mxf4)
-// leave less than ~2^-18 (E4M3) / ~2^-16 (E2M1) of the block's largest
-// element; the error of the dot products is below 1e-4 relative, far under
-// the FFN tolerance.  Both encoders are warp-cooperative: lane l holds
-// element l of one 32-element block.
+// as a short sum of narrow terms, v = sum_t 2^(s_t) * c_t, term t encoding
+// what terms 0..t-1 left over.
+//  * kind::mxf8f6f4: two E4M3 terms with an E8M0 scale per 32 elements
+//    (what is lost is below ~2^-18 of the block's largest element);
+//    warp-cooperative, lane l holds element l of one 32-element block.
+//  * kind::mxf4: four E2M1 terms with ONE scale per row and term, chosen
+//    from the row's largest remaining magnitude.  The MMA then sees a
+//    constant block scale of 1.0 for B (copied to tensor memory once per
+//    CTA), and the epilogue multiplies each term's column by its exact power
+//    of two.  Four terms leave ~1e-4 relative error in the dot products.
 
 
 __device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(127 + s) << 23); }
@@ -259,24 +262,6 @@ __device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t
   }
 }
 
-// Four E2M1 terms: 4-bit codes q[0..3] of this lane, scale bytes sb[0..3].
-__device__ __forceinline__ void encode_e2m1x4(float v, uint32_t (&q)[4], uint8_t (&sb)[4]) {
-  float r = v;
-#pragma unroll
-  for (int t = 0; t < 4; ++t) {
-    const float amax = warp_max(fabsf(r));
-    int s = 0;
-    uint32_t c = 0;
-    if (amax > 0.f) {
-      s = e2m1_block_exp(amax);
-      c = to_e2m1(r * pow2f(-s));
-      r -= e2m1x2_to_f32x2(c).x * pow2f(s);
-    }
-    q[t] = c;
-    sb[t] = (uint8_t)(127 + s);
-  }
-}
-
 // Kind of tensor-core MMA used by the FFN.
 enum TcKind { KIND_F8 = 0, KIND_F4 = 1 };
 
@@ -288,40 +273,27 @@ struct TcKindCfg {
   static constexpr int kMmaK = kStageK / 4;                     // 4 MMAs per stage
   static constexpr uint32_t kABytes = 128u * kStageK / 2;       // packed weight bytes per stage
   static constexpr int kBRowBytesPerK2 = KIND == KIND_F4 ? 1 : 2;  // B row bytes = K * this / 2
+  static constexpr bool kRowScaledB = KIND == KIND_F4;          // B scales per row, not block
 };
 
-// Stores one lane's encoded element n of activation row r (terms in rows
-// T*r + t) and the block's scale bytes.
-template <int KIND>
-__device__ __forceinline__ void store_terms(float v, size_t r, int n, int kdim, uint8_t *q_out,
-                                            uint8_t *s_out, int lane, bool valid) {
-  if (KIND == KIND_F4) {
-    uint32_t q[4];
-    uint8_t sb[4];
-    encode_e2m1x4(v, q, sb);
+// Stores one lane's two E4M3 terms of element n of activation row r (B rows
+// 2r, 2r+1) and, from lane 0, the block's two scale bytes.
+__device__ __forceinline__ void store_terms_f8(float v, size_t r, int n, int kdim,
+                                               uint8_t *q_out, uint8_t *s_out, int lane,
+                                               bool valid) {
+  uint32_t q[2];
+  uint8_t sb[2];
+  encode_e4m3x2(v, q, sb);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const uint32_t hi = __shfl_down_sync(FULL, q[t], 1);
-      if (valid && !(lane & 1))
-        q_out[(4 * r + t) * (size_t)(kdim / 2) + n / 2] = (uint8_t)(q[t] | (hi << 4));
-      if (valid && lane == 0) s_out[(4 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
-    }
-  } else {
-    uint32_t q[2];
-    uint8_t sb[2];
-    encode_e4m3x2(v, q, sb);
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      if (valid) q_out[(2 * r + t) * (size_t)kdim + n] = (uint8_t)q[t];
-      if (valid && lane == 0) s_out[(2 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
-    }
+  for (int t = 0; t < 2; ++t) {
+    if (valid) q_out[(2 * r + t) * (size_t)kdim + n] = (uint8_t)q[t];
+    if (valid && lane == 0) s_out[(2 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
   }
 }
 
-// Activation operand of GEMM-1: for every sorted row r (token sp[r]/k) the
-// terms of x[token] as B rows T*r + t, and their scale bytes.  One warp per
-// 32-element block.
-template <int KIND>
+// kind::mxf8f6f4 activation operand of GEMM-1: for every sorted row r (token
+// sp[r]/k) the two E4M3 terms of x[token] as B rows 2r, 2r+1, and their scale
+// bytes.  One warp per 32-element block.
 __global__ void __launch_bounds__(256)
 split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, int P, int k,
                int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
@@ -333,7 +305,60 @@ split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, i
     const int r = (int)(w / nb), b = (int)(w % nb);
     const int t = __ldg(sp + r) / k;
     const float v = __uint_as_float((uint32_t)__ldg(x + (size_t)t * H + b * 32 + lane) << 16);
-    store_terms<KIND>(v, (size_t)r, b * 32 + lane, H, xq, xs, lane, true);
+    store_terms_f8(v, (size_t)r, b * 32 + lane, H, xq, xs, lane, true);
+  }
+}
+
+// kind::mxf4 activation operand: row r of the source (x[sp[r]/k] when sp is
+// given, else src row r) as four E2M1 terms, B rows 4r..4r+3 (packed, K/2
+// bytes each), and the four per-row scales 2^(s_t) as floats.  One CTA per
+// row; each thread keeps its elements (pairs 2i, 2i+1 for i = tid + 256j) in
+// registers; K <= 2 * 256 * ENC_MAX_PAIRS.
+constexpr int ENC_THREADS = 256;
+constexpr int ENC_MAX_PAIRS = 16;
+
+__global__ void __launch_bounds__(ENC_THREADS)
+encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp, int k,
+                      int K, uint8_t *__restrict__ q, float *__restrict__ rs) {
+  const int r = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const uint16_t *row = src + (size_t)(sp ? __ldg(sp + r) / k : r) * K;
+  __shared__ float red[ENC_THREADS / 32];
+  const int npairs = K / 2;
+  float v[2 * ENC_MAX_PAIRS];
+#pragma unroll
+  for (int j = 0; j < ENC_MAX_PAIRS; ++j) {
+    const int i = tid + ENC_THREADS * j;
+    uint32_t pr = 0;
+    if (i < npairs) pr = __ldg(reinterpret_cast<const uint32_t *>(row) + i);
+    v[2 * j] = bf16_lo(pr);
+    v[2 * j + 1] = bf16_hi(pr);
+  }
+#pragma unroll 1
+  for (int t = 0; t < 4; ++t) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2 * ENC_MAX_PAIRS; ++j) m = fmaxf(m, fabsf(v[j]));
+    m = warp_max(m);
+    __syncthreads();                       // red[] reuse across terms
+    if (lane == 0) red[w] = m;
+    __syncthreads();
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < ENC_THREADS / 32; ++i) amax = fmaxf(amax, red[i]);
+    const int sexp = amax > 0.f ? e2m1_block_exp(amax) : 0;
+    const float inv = pow2f(-sexp), sc = pow2f(sexp);
+    uint8_t *qrow = q + (size_t)(4 * r + t) * (K / 2);
+#pragma unroll
+    for (int j = 0; j < ENC_MAX_PAIRS; ++j) {
+      const int i = tid + ENC_THREADS * j;
+      const uint32_t c0 = to_e2m1(v[2 * j] * inv), c1 = to_e2m1(v[2 * j + 1] * inv);
+      const float2 d = e2m1x2_to_f32x2(c0 | (c1 << 4));
+      v[2 * j] -= d.x * sc;
+      v[2 * j + 1] -= d.y * sc;
+      if (i < npairs) qrow[i] = (uint8_t)(c0 | (c1 << 4));
+    }
+    if (tid == 0) rs[4 * r + t] = sc;
   }
 }
 
@@ -346,7 +371,8 @@ struct TcMaps {
 
 struct TcArgs {
   const uint8_t *a_scales;   // [E*rows, K/32]
-  const uint8_t *b_scales;   // [T*P, K/32]
+  const uint8_t *b_scales;   // kind::mxf8f6f4: [T*P, K/32] block scale bytes
+  const float *b_rowscale;   // kind::mxf4: [T*P] per-row, per-term scales
   const int32_t *off;        // [E+1]
   int E, K, rows_per_expert, P;
   int I;                     // GEMM-1: the gate/up split
@@ -367,19 +393,22 @@ struct TcCfg {
   static constexpr int kA = 128 * 128;                              // smem bytes of one A stage
   static constexpr int kB = BN * 128;
   static constexpr int kSfa = 512 * Kd::kKGroups;
-  static constexpr int kSfb = 512 * Kd::kKGroups * kRowChunks;
+  static constexpr int kSfb = Kd::kRowScaledB ? 0 : 512 * Kd::kKGroups * kRowChunks;
+  static constexpr int kSfbConst = Kd::kRowScaledB ? 512 * kRowChunks : 0;  // all 1.0
   static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
-  static constexpr int kFixed = 1024 + 2048 + 2 * 1025 * 4 + 1024;  // barriers, xchg, table, slack
+  static constexpr int kFixed = 1024 + 2048 + 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
   static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
   static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
-  static constexpr int kSfCols = 4 * Kd::kKGroups * (1 + kRowChunks);   // TMEM columns per stage
+  static constexpr int kSfCols =                                    // TMEM columns per stage
+      4 * Kd::kKGroups * (Kd::kRowScaledB ? 1 : 1 + kRowChunks);
   static constexpr int kAcc = BN <= 128 ? 2 : 1;                   // accumulator buffers
   // Independent accumulation chains per buffer: with few B columns each MMA
   // is tiny and a single chain would run at MMA latency; MMA kk of a stage
   // accumulates into chain kk % kChains and the epilogue adds the chains.
   static constexpr int kChains = BN <= 32 ? 4 : BN <= 64 ? 2 : 1;
   static constexpr int kAccCols = kAcc * kChains * BN;
-  static constexpr int kUsed = kAccCols + kStages * kSfCols;
+  static constexpr int kSfbConstCols = Kd::kRowScaledB ? 4 * kRowChunks : 0;
+  static constexpr int kUsed = kAccCols + kStages * kSfCols + kSfbConstCols;
   static constexpr int kTmemCols = kUsed <= 128 ? 128 : kUsed <= 256 ? 256 : 512;
   static_assert(kUsed <= 512, "TMEM budget");
   static constexpr int kOffB = kStages * kA;
@@ -388,8 +417,11 @@ struct TcCfg {
   static constexpr int kOffBar = kOffSfb + kStages * kSfb;
   static constexpr int kOffXchg = kOffBar + 1024;                // 64 rows x 4 tokens (float)
   static constexpr int kOffTab = kOffXchg + 2048;                 // active list + prefix
-  static constexpr int kSmem = kOffTab + 2 * 1025 * 4 + 1024;     // + alignment slack
+  static constexpr int kOffSfbConst = (kOffTab + 2 * 1025 * 4 + 127) & ~127;  // 16B-aligned for tcgen05.cp
+  static constexpr int kSmem = kOffSfbConst + kSfbConst + 1024;   // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
+  static_assert(kOffSfa % 1024 == 0 && kOffSfb % 128 == 0 && kOffSfbConst % 128 == 0,
+                "descriptor alignment");
 };
 
 constexpr int TC_THREADS = 256;
@@ -458,6 +490,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                      smem_u32(tmem_slot)),
                  "r"(C::kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (Kd::kRowScaledB && warp == 3) {
+    // constant B block scales (byte 127 = 1.0), copied to tensor memory once
+    uint32_t *cst = reinterpret_cast<uint32_t *>(smem + C::kOffSfbConst);
+    for (int i = lane; i < C::kSfbConst / 4; i += 32) cst[i] = 0x7f7f7f7fu;
+    fence_proxy_async();
   }
   tc_fence_before();
   __syncthreads();
@@ -553,7 +591,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 #pragma unroll
           for (int q = 0; q < 4 * C::kRowChunks; ++q) {
             const int i = lane + 32 * q;
-            if (i < nB)
+            if (!Kd::kRowScaledB && i < nB)
               cp_async4(sfb + 512 * (g * C::kRowChunks + (q >> 2)) + 16 * lane + 4 * (q & 3),
                         a.b_scales + (size_t)(rowB + i) * kb + koff);
           }
@@ -569,6 +607,14 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       int stage = 0;
       uint32_t phase = 0;
       const uint32_t sf_col0 = (uint32_t)C::kAccCols;
+      const uint32_t sfb_const_t = tmem + sf_col0 + C::kStages * C::kSfCols;
+      if (Kd::kRowScaledB) {
+#pragma unroll
+        for (int c = 0; c < C::kRowChunks; ++c)
+          tc_cp_32x128b(sfb_const_t + 4 * c,
+                        smem_desc(smem_u32(smem + C::kOffSfbConst + 512 * c), 0, 128,
+                                  kSwizzleNone));
+      }
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
         int e, mt, rowB, nB;
@@ -594,6 +640,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 #pragma unroll
           for (int g = 0; g < Kd::kKGroups; ++g) {
             tc_cp_32x128b(sfa_t + 4 * g, smem_desc(sa + 512 * g, 0, 128, kSwizzleNone));
+            if (!Kd::kRowScaledB)
 #pragma unroll
             for (int c = 0; c < C::kRowChunks; ++c)
               tc_cp_32x128b(sfb_t + 4 * (g * C::kRowChunks + c),
@@ -612,8 +659,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
               const int g = kk >> 1;                     // scale group of this MMA
               const uint32_t sfid = 2u * (kk & 1);      // two scale bytes per row
               mma_mxf4(d_t, ad, bd, idesc_block_scaled(1, 1, ncol, sfid),
-                       (sfa_t + 4 * g) | (sfid << 30),
-                       (sfb_t + 4 * g * C::kRowChunks) | (sfid << 30), acc);
+                       (sfa_t + 4 * g) | (sfid << 30), sfb_const_t | (sfid << 30), acc);
             } else {
               mma_mxf8f6f4(d_t, ad, bd, idesc_block_scaled(5, 0, ncol, kk),
                            sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30), acc);
@@ -653,15 +699,22 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += w[i];
         }
+        const int tok0 = c0 / T;
         float tok_sum[kTokPerLd];
 #pragma unroll
         for (int j = 0; j < kTokPerLd; ++j) {
           float sum = 0.f;
+          if (Kd::kRowScaledB) {
+            const int tok = min(tok0 + j, ntok - 1);     // rows past ntok are discarded
+            const float *rsc = a.b_rowscale + (size_t)(rtok0 + tok) * T;
 #pragma unroll
-          for (int u = 0; u < T; ++u) sum += v[T * j + u];
+            for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], __ldg(rsc + u), sum);
+          } else {
+#pragma unroll
+            for (int u = 0; u < T; ++u) sum += v[T * j + u];
+          }
           tok_sum[j] = sum;
         }
-        const int tok0 = c0 / T;
         if (MODE == 2) {
           const int m = mt * 128 + 32 * q + lane;
 #pragma unroll
@@ -685,8 +738,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
               const bool valid = tok < ntok;
               const size_t r = (size_t)(rtok0 + tok);
               if (valid) a.h[r * a.I + n] = hb;
-              store_terms<KIND>(__uint_as_float((uint32_t)hb << 16), r, n, a.I, a.hq, a.hs,
-                                lane, valid);
+              if (!Kd::kRowScaledB)     // kind::mxf4 encodes h rows in a separate pass
+                store_terms_f8(__uint_as_float((uint32_t)hb << 16), r, n, a.I, a.hq, a.hs,
+                               lane, valid);
             }
           }
           asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -794,10 +848,13 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
     cudaFuncSetAttribute(tc_gemm_kernel<KIND, 2, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          C::kSmem);
   }
-  {
+  if (KIND == KIND_F4) {
+    encode_rows_f4_kernel<<<(unsigned)P, ENC_THREADS, 0, s>>>(f.x, f.sp, f.k, H, xq,
+                                                             reinterpret_cast<float *>(xs));
+  } else {
     const long blocks = (long)P * (H / 32);
     const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
-    split_x_kernel<KIND><<<grid, 256, 0, s>>>(f.x, f.sp, (int)P, f.k, H, xq, xs);
+    split_x_kernel<<<grid, 256, 0, s>>>(f.x, f.sp, (int)P, f.k, H, xq, xs);
   }
   TcMaps maps;
   TcArgs a{};
@@ -820,11 +877,15 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
   a.a_scales = f.w13s;
   a.b_scales = xs;
+  a.b_rowscale = reinterpret_cast<const float *>(xs);
   a.K = H;
   a.rows_per_expert = 2 * I;
   tc_gemm_kernel<KIND, 1, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
+  if (KIND == KIND_F4)
+    encode_rows_f4_kernel<<<(unsigned)P, ENC_THREADS, 0, s>>>(f.h, nullptr, 1, I, hq,
+                                                             reinterpret_cast<float *>(hs));
   // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
   for (int i = 0; i < 5; ++i)
@@ -833,6 +894,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
   a.a_scales = f.w2s;
   a.b_scales = hs;
+  a.b_rowscale = reinterpret_cast<const float *>(hs);
   a.K = I;
   a.rows_per_expert = H;
   tc_gemm_kernel<KIND, 2, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
@@ -857,9 +919,15 @@ inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
 // stages, else kind::mxf8f6f4.
 inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int kind) {
   if (f.H < 512 || f.I < 128) return MOE_ERR_UNSUPPORTED;   // scale rows of >= 16 bytes
-  if (kind < 0) kind = (f.H % 256 == 0 && f.I % 256 == 0) ? KIND_F4 : KIND_F8;
+  if (kind < 0)
+    kind = (f.H % 256 == 0 && f.I % 256 == 0 && f.H <= 2 * ENC_THREADS * ENC_MAX_PAIRS &&
+            f.I <= 2 * ENC_THREADS * ENC_MAX_PAIRS)
+               ? KIND_F4
+               : KIND_F8;
   if (kind == KIND_F4) {
-    if (f.H % 256 || f.I % 256) return MOE_ERR_UNSUPPORTED;
+    if (f.H % 256 || f.I % 256 || f.H > 2 * ENC_THREADS * ENC_MAX_PAIRS ||
+        f.I > 2 * ENC_THREADS * ENC_MAX_PAIRS)
+      return MOE_ERR_UNSUPPORTED;
     return tc_dispatch<KIND_F4>(f, ws, sms, s);
   }
   return tc_dispatch<KIND_F8>(f, ws, sms, s);

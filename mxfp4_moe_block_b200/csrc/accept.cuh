@@ -55,19 +55,32 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
 #pragma unroll
     for (int r = 0; r < GREEDY_ROWS; ++r) { bv[r] = 0.f; bi[r] = -1; }
     if (vec) {
-      for (int u = u0 + threadIdx.x; u < u1; u += blockDim.x) {
-        float4 q[GREEDY_ROWS];
-#pragma unroll
-        for (int r = 0; r < GREEDY_ROWS; ++r)
-          if (r < nr) q[r] = __ldcs(reinterpret_cast<const float4 *>(rows + (size_t)r * V) + u);
+      // two strided units per iteration: 2 x 8 independent 16-byte loads in
+      // flight per thread (the lowest-index rule makes the order irrelevant)
+      const int step = blockDim.x;
+      for (int u = u0 + threadIdx.x; u < u1; u += 2 * step) {
+        const int u2 = u + step;
+        float4 q[2][GREEDY_ROWS];
 #pragma unroll
         for (int r = 0; r < GREEDY_ROWS; ++r) {
-          if (r < nr) {
-            const int b = 4 * u;
-            if (better(q[r].x, b, bv[r], bi[r])) { bv[r] = q[r].x; bi[r] = b; }
-            if (better(q[r].y, b + 1, bv[r], bi[r])) { bv[r] = q[r].y; bi[r] = b + 1; }
-            if (better(q[r].z, b + 2, bv[r], bi[r])) { bv[r] = q[r].z; bi[r] = b + 2; }
-            if (better(q[r].w, b + 3, bv[r], bi[r])) { bv[r] = q[r].w; bi[r] = b + 3; }
+          const float4 *rp = reinterpret_cast<const float4 *>(rows + (size_t)r * V);
+          if (r < nr) q[0][r] = __ldcs(rp + u);
+          if (r < nr && u2 < u1) q[1][r] = __ldcs(rp + u2);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int uu = h ? u2 : u;
+          if (h && uu >= u1) break;
+#pragma unroll
+          for (int r = 0; r < GREEDY_ROWS; ++r) {
+            if (r < nr) {
+              const int b = 4 * uu;
+              const float4 qq = q[h][r];
+              if (better(qq.x, b, bv[r], bi[r])) { bv[r] = qq.x; bi[r] = b; }
+              if (better(qq.y, b + 1, bv[r], bi[r])) { bv[r] = qq.y; bi[r] = b + 1; }
+              if (better(qq.z, b + 2, bv[r], bi[r])) { bv[r] = qq.z; bi[r] = b + 2; }
+              if (better(qq.w, b + 3, bv[r], bi[r])) { bv[r] = qq.w; bi[r] = b + 3; }
+            }
           }
         }
       }

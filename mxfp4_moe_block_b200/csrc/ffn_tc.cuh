@@ -264,10 +264,11 @@ __device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t
 
 // Kind of tensor-core MMA used by the FFN.
 enum TcKind { KIND_F8 = 0, KIND_F4 = 1 };
+constexpr int kF4Terms = 8;     // E2M1 terms per activation row (kind::mxf4)
 
 template <int KIND>
 struct TcKindCfg {
-  static constexpr int kTerms = KIND == KIND_F4 ? 4 : 2;        // B rows per token
+  static constexpr int kTerms = KIND == KIND_F4 ? kF4Terms : 2;  // B rows per token
   static constexpr int kStageK = KIND == KIND_F4 ? 256 : 128;   // K elements per stage
   static constexpr int kKGroups = kStageK / 128;                // 4-scale groups per stage
   static constexpr int kMmaK = kStageK / 4;                     // 4 MMAs per stage
@@ -310,13 +311,14 @@ split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, i
 }
 
 // kind::mxf4 activation operand: row r of the source (x[sp[r]/k] when sp is
-// given, else src row r) as four E2M1 terms, B rows 4r..4r+3 (packed, K/2
-// bytes each), and the four per-row scales 2^(s_t) as floats.  One CTA per
+// given, else src row r) as NT E2M1 terms, B rows NT*r + t (packed, K/2
+// bytes each), and the NT per-row scales 2^(s_t) as floats.  One CTA per
 // row; each thread keeps its elements (pairs 2i, 2i+1 for i = tid + 256j) in
 // registers; K <= 2 * 256 * ENC_MAX_PAIRS.
 constexpr int ENC_THREADS = 256;
 constexpr int ENC_MAX_PAIRS = 16;
 
+template <int NT>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp, int k,
                       int K, uint8_t *__restrict__ q, float *__restrict__ rs) {
@@ -335,7 +337,7 @@ encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restric
     v[2 * j + 1] = bf16_hi(pr);
   }
 #pragma unroll 1
-  for (int t = 0; t < 4; ++t) {
+  for (int t = 0; t < NT; ++t) {
     float m = 0.f;
 #pragma unroll
     for (int j = 0; j < 2 * ENC_MAX_PAIRS; ++j) m = fmaxf(m, fabsf(v[j]));
@@ -348,7 +350,7 @@ encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restric
     for (int i = 0; i < ENC_THREADS / 32; ++i) amax = fmaxf(amax, red[i]);
     const int sexp = amax > 0.f ? e2m1_block_exp(amax) : 0;
     const float inv = pow2f(-sexp), sc = pow2f(sexp);
-    uint8_t *qrow = q + (size_t)(4 * r + t) * (K / 2);
+    uint8_t *qrow = q + (size_t)(NT * r + t) * (K / 2);
 #pragma unroll
     for (int j = 0; j < ENC_MAX_PAIRS; ++j) {
       const int i = tid + ENC_THREADS * j;
@@ -358,7 +360,7 @@ encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restric
       v[2 * j + 1] -= d.y * sc;
       if (i < npairs) qrow[i] = (uint8_t)(c0 | (c1 << 4));
     }
-    if (tid == 0) rs[4 * r + t] = sc;
+    if (tid == 0) rs[NT * r + t] = sc;
   }
 }
 
@@ -764,11 +766,20 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
 
 inline size_t align256_tc(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Operands of either kind: terms of x [T*P, H bytes*] and of h, plus scales
-// for up to 4 terms per row.
+// Operands of either kind: the terms of x and of h (kind::mxf8f6f4: 2 rows of
+// K bytes per sorted row; kind::mxf4: kTerms rows of K/2 bytes) and their
+// scales (block scale bytes [2P, K/32], or kTerms floats per row).
+inline size_t tc_term_bytes(size_t P, int K) {
+  const size_t f8 = 2 * P * (size_t)K, f4 = kF4Terms * P * (size_t)K / 2;
+  return f8 > f4 ? f8 : f4;
+}
+inline size_t tc_scale_bytes(size_t P, int K) {
+  const size_t f8 = 2 * P * (size_t)K / 32, f4 = kF4Terms * P * sizeof(float);
+  return f8 > f4 ? f8 : f4;
+}
 inline size_t tc_workspace_bytes(size_t P, int H, int I) {
-  return align256_tc(2 * P * H) + align256_tc(4 * P * H / 32) + align256_tc(2 * P * I) +
-         align256_tc(4 * P * I / 32);
+  return align256_tc(tc_term_bytes(P, H)) + align256_tc(tc_scale_bytes(P, H)) +
+         align256_tc(tc_term_bytes(P, I)) + align256_tc(tc_scale_bytes(P, I));
 }
 
 // The tensor-core variant streams the weights with TMA and needs no
@@ -834,9 +845,9 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   const size_t xrow = (size_t)H * Kd::kBRowBytesPerK2 / 2;   // bytes per term row of x
   const size_t hrow = (size_t)I * Kd::kBRowBytesPerK2 / 2;
   uint8_t *xq = ws;
-  uint8_t *xs = xq + align256_tc(2 * P * H);
-  uint8_t *hq = xs + align256_tc(4 * P * H / 32);
-  uint8_t *hs = hq + align256_tc(2 * P * I);
+  uint8_t *xs = xq + align256_tc(tc_term_bytes(P, H));
+  uint8_t *hq = xs + align256_tc(tc_scale_bytes(P, H));
+  uint8_t *hs = hq + align256_tc(tc_term_bytes(P, I));
 
   int dev = 0;
   cudaGetDevice(&dev);
@@ -849,8 +860,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
                          C::kSmem);
   }
   if (KIND == KIND_F4) {
-    encode_rows_f4_kernel<<<(unsigned)P, ENC_THREADS, 0, s>>>(f.x, f.sp, f.k, H, xq,
-                                                             reinterpret_cast<float *>(xs));
+    encode_rows_f4_kernel<T><<<(unsigned)P, ENC_THREADS, 0, s>>>(f.x, f.sp, f.k, H, xq,
+                                                                reinterpret_cast<float *>(xs));
   } else {
     const long blocks = (long)P * (H / 32);
     const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
@@ -884,8 +895,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
 
   if (KIND == KIND_F4)
-    encode_rows_f4_kernel<<<(unsigned)P, ENC_THREADS, 0, s>>>(f.h, nullptr, 1, I, hq,
-                                                             reinterpret_cast<float *>(hs));
+    encode_rows_f4_kernel<T><<<(unsigned)P, ENC_THREADS, 0, s>>>(f.h, nullptr, 1, I, hq,
+                                                                reinterpret_cast<float *>(hs));
   // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
   for (int i = 0; i < 5; ++i)

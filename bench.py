@@ -90,6 +90,35 @@ def load_traffic(workload, variant_name):
         return None
 
 
+def workload_config(sh, world):
+    """The `config` object of the JSON line (identical for both arms)."""
+    acc = " + ".join(sh.accept)
+    layers = f"{sh.layers} stacked MoE layers" if sh.layers > 1 else "one MoE layer"
+    return {
+        "workload": f"{sh.name}: {layers} H={sh.H} I={sh.I} E={sh.E} top-{sh.k} SwiGLU, "
+                    f"S={sh.S} x K={sh.K} block, {acc} acceptance over V={sh.V}",
+        "global_batch_tokens": sh.T * world,
+        "parallelism": f"replicas x{world} (independent batches, no collective)",
+        "l2": "inputs larger than L2: >= 1 GB of MXFP4 expert weights read per step",
+    }
+
+
+def rank_shape(sh, rank):
+    """Each rank verifies its own batch: same weights, different activations,
+    router logits and drafts."""
+    return synth.Shape(**{**sh.__dict__, "seed": sh.seed + 7919 * rank})
+
+
+def max_over_ranks(value, world, device):
+    """Slowest rank's value (all-reduce MAX); identity on one rank."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -150,8 +179,7 @@ class Workload:
         self.mm = mm
         self.sh = sh
         self.dev = device
-        # every rank verifies its own batch: different activations / logits
-        self.sh_r = synth.Shape(**{**sh.__dict__, "seed": sh.seed + 7919 * rank})
+        self.sh_r = rank_shape(sh, rank)
         s = self.sh_r
         self.x_bits = synth.x_bf16_bits(s)
         self.logits_np = synth.router_logits(s)
@@ -199,6 +227,19 @@ class Workload:
 
     def ffn_flops(self):
         return 2.0 * self.sh_r.P * 3 * self.sh.H * self.sh.I
+
+
+def count_launches(wl, variant):
+    """Kernels one eager step launches, counted by the CUDA profiler (CUPTI)."""
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        wl.step(variant)
+        torch.cuda.synchronize()
+    names = [ev.name for ev in prof.events()
+             if ev.device_type == torch.autograd.DeviceType.CUDA
+             and not ev.name.lower().startswith(("memcpy", "memset"))]
+    return len(names), sorted(set(names))
 
 
 def e2e_time(wl, variant, steps, warmup):
@@ -302,8 +343,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded counter-based generator)",
-            "config": {"workload": f"{sh.name}: H={sh.H} I={sh.I} E={sh.E} top-{sh.k}, "
-                                   f"S={sh.S} x K={sh.K}, V={sh.V}"},
+            "config": workload_config(sh, 1),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"route+permute+combine+greedy in full; expert FFN on "
                                        f"{info['experts_sampled']} of {info['experts_active']} "
@@ -381,37 +421,27 @@ def main():
     ffn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     tail_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
     else:
         e2e_ms, h2d, d2h = e2e_time(wl, variant, args.steps, 3)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     peak, peak_kind = load_peaks()
     achieved = act_bytes / (ffn_ms * 1e-3) / 1e9
     vname = {0: "auto", 1: "fma", 2: "tensor"}[variant]
     traffic = load_traffic(sh.name, vname)
     tokens = sh.T * world
-    # route, permute, FFN (3 kernels), combine, greedy
-    launches_per_step = 7
+    launches_per_step, kernel_names = count_launches(wl, variant)
     line = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4 weights, bf16 activations, f32 accumulate",
         "data": "synthetic (seeded counter-based generator; random MXFP4 weights)",
-        "config": {"workload": f"{sh.name}: one MoE layer H={sh.H} I={sh.I} E={sh.E} top-{sh.k} SwiGLU, "
-                               f"S={sh.S} x K={sh.K} block, greedy over V={sh.V}",
-                   "global_batch_tokens": tokens, "parallelism": f"replicas x{world} (independent batches)",
-                   "l2": "inputs larger than L2: %.2f GB of expert weights read per step" % (act_bytes / 1e9),
-                   "ffn_variant": vname, "timing": "CUDA graph replay" if graph is not None else "eager"},
+        "config": workload_config(sh, world),
+        "ffn_variant": vname, "timing": "CUDA graph replay" if graph is not None else "eager",
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "mxfp4_moe_ffn (GEMM-1+SwiGLU and GEMM-2 launches)",
@@ -423,6 +453,8 @@ def main():
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "launches_per_step": launches_per_step,
+        "kernels": [n.split("(")[0].split("<")[0].replace("void ", "") for n in kernel_names],
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -917,8 +917,11 @@ template <int KIND>
 inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   const size_t P = (size_t)f.T * f.k;
   const size_t used = P < (size_t)f.E ? P : (size_t)f.E;
-  const size_t rows = (TcKindCfg<KIND>::kTerms * P + used - 1) / used;  // B rows per expert
-  const size_t want = rows + rows / 2;
+  const size_t terms = TcKindCfg<KIND>::kTerms;
+  const size_t rows = (terms * P + used - 1) / used;           // B rows per expert, average
+  // room for the busier experts, and at least 4 tokens per B tile
+  size_t want = rows + rows / 2;
+  if (want < 4 * terms) want = 4 * terms;
   if (want <= 16) return tc_run<KIND, 16>(f, ws, sms, s);
   if (want <= 32) return tc_run<KIND, 32>(f, ws, sms, s);
   if (want <= 64) return tc_run<KIND, 64>(f, ws, sms, s);
@@ -930,11 +933,19 @@ inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
 // stages, else kind::mxf8f6f4.
 inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int kind) {
   if (f.H < 512 || f.I < 128) return MOE_ERR_UNSUPPORTED;   // scale rows of >= 16 bytes
-  if (kind < 0)
-    kind = (f.H % 256 == 0 && f.I % 256 == 0 && f.H <= 2 * ENC_THREADS * ENC_MAX_PAIRS &&
-            f.I <= 2 * ENC_THREADS * ENC_MAX_PAIRS)
-               ? KIND_F4
-               : KIND_F8;
+  if (kind < 0) {
+    // kind::mxf4 (exact 8-term activations) while the B tiles stay narrow --
+    // at small N the extra term columns cost nothing; with many tokens per
+    // expert the 8 terms double the MMA work and kind::mxf8f6f4 (two E4M3
+    // terms) is faster.
+    const size_t P = (size_t)f.T * f.k;
+    const size_t used = P < (size_t)f.E ? P : (size_t)f.E;
+    const bool narrow = (size_t)kF4Terms * P <= 128 * used;
+    const bool f4_ok = f.H % 256 == 0 && f.I % 256 == 0 &&
+                       f.H <= 2 * ENC_THREADS * ENC_MAX_PAIRS &&
+                       f.I <= 2 * ENC_THREADS * ENC_MAX_PAIRS;
+    kind = (f4_ok && narrow) ? KIND_F4 : KIND_F8;
+  }
   if (kind == KIND_F4) {
     if (f.H % 256 || f.I % 256 || f.H > 2 * ENC_THREADS * ENC_MAX_PAIRS ||
         f.I > 2 * ENC_THREADS * ENC_MAX_PAIRS)

@@ -19,19 +19,35 @@
 namespace moe {
 namespace cg = cooperative_groups;
 
-constexpr int GREEDY_THREADS = 512;
-constexpr int GREEDY_ROWS = 8;       // rows scanned together: 8 independent loads in flight
+constexpr int GREEDY_MAX_THREADS = 1024;
+constexpr int GREEDY_ROWS = 4;       // rows scanned together
 constexpr int GREEDY_CLUSTER = 16;   // CTAs per sequence (non-portable cluster size)
 
-// grid (cluster_size, S), cluster (cluster_size, 1, 1).  CTA r of a
-// sequence's cluster owns slice r of [0, V) of every row; a thread walks its
-// units of that slice for up to 8 rows at once, keeping one (value, index)
-// candidate per row; warps, then the CTA, then the cluster (through
-// distributed shared memory) reduce them with the lowest-index tie rule.
-__global__ void __launch_bounds__(GREEDY_THREADS)
+// One 16-byte unit of a row (elements b..b+3), visited in increasing index
+// order by this thread: the running (bv, bi) keeps the first occurrence of
+// the largest value.  The max of the four is one comparison away from the
+// running best, and the index search runs only when the best improves.
+__device__ __forceinline__ void scan_unit(const float4 q, int b, float &bv, int &bi) {
+  const float m = fmaxf(fmaxf(q.x, q.y), fmaxf(q.z, q.w));
+  if (m > bv) {
+    bv = m;
+    bi = q.x == m ? b : q.y == m ? b + 1 : q.z == m ? b + 2 : b + 3;
+  }
+}
+
+// grid (cluster_size, S), cluster (cluster_size, 1, 1), blockDim a multiple
+// of 32 up to 1024.  CTA r of a sequence's cluster owns slice r of [0, V) of
+// every row; a thread walks its units of that slice for up to 8 rows at once
+// in increasing index order, keeping one (value, index) candidate per row;
+// warps, then the CTA, then the cluster (through distributed shared memory)
+// reduce the candidates with the lowest-index tie rule.  Rows hold finite
+// values (a row of -inf has no candidate and never matches a draft).
+__global__ void __launch_bounds__(GREEDY_MAX_THREADS, 1)
 greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draft,
               int S, int K, int V, int32_t *__restrict__ accept_len,
               int32_t *__restrict__ next_token) {
+  pdl_wait();
+  pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int ncta = (int)cluster.num_blocks();
@@ -39,8 +55,8 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   __shared__ float part_v[32];
   __shared__ int part_i[32];
-  __shared__ float red_v[GREEDY_THREADS / 32][32];
-  __shared__ int red_i[GREEDY_THREADS / 32][32];
+  __shared__ float red_v[GREEDY_MAX_THREADS / 32][32];
+  __shared__ int red_i[GREEDY_MAX_THREADS / 32][32];
 
   const bool vec = (V & 3) == 0;       // rows 16-byte aligned: float4 units
   const int units = vec ? V / 4 : V;
@@ -53,35 +69,28 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
     float bv[GREEDY_ROWS];
     int bi[GREEDY_ROWS];
 #pragma unroll
-    for (int r = 0; r < GREEDY_ROWS; ++r) { bv[r] = 0.f; bi[r] = -1; }
+    for (int r = 0; r < GREEDY_ROWS; ++r) { bv[r] = -INFINITY; bi[r] = -1; }
     if (vec) {
-      // two strided units per iteration: 2 x 8 independent 16-byte loads in
-      // flight per thread (the lowest-index rule makes the order irrelevant)
+      // two strided units per iteration: 2 x GREEDY_ROWS independent
+      // 16-byte loads in flight per thread, consumed in index order
+      const float4 *rows4 = reinterpret_cast<const float4 *>(rows);
       const int step = blockDim.x;
       for (int u = u0 + threadIdx.x; u < u1; u += 2 * step) {
         const int u2 = u + step;
         float4 q[2][GREEDY_ROWS];
 #pragma unroll
         for (int r = 0; r < GREEDY_ROWS; ++r) {
-          const float4 *rp = reinterpret_cast<const float4 *>(rows + (size_t)r * V);
-          if (r < nr) q[0][r] = __ldcs(rp + u);
-          if (r < nr && u2 < u1) q[1][r] = __ldcs(rp + u2);
+          const float4 *p = rows4 + (size_t)r * units;
+          if (r < nr) q[0][r] = __ldcs(p + u);
+          if (r < nr && u2 < u1) q[1][r] = __ldcs(p + u2);
         }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int uu = h ? u2 : u;
-          if (h && uu >= u1) break;
+        for (int r = 0; r < GREEDY_ROWS; ++r)
+          if (r < nr) scan_unit(q[0][r], 4 * u, bv[r], bi[r]);
+        if (u2 < u1) {
 #pragma unroll
-          for (int r = 0; r < GREEDY_ROWS; ++r) {
-            if (r < nr) {
-              const int b = 4 * uu;
-              const float4 qq = q[h][r];
-              if (better(qq.x, b, bv[r], bi[r])) { bv[r] = qq.x; bi[r] = b; }
-              if (better(qq.y, b + 1, bv[r], bi[r])) { bv[r] = qq.y; bi[r] = b + 1; }
-              if (better(qq.z, b + 2, bv[r], bi[r])) { bv[r] = qq.z; bi[r] = b + 2; }
-              if (better(qq.w, b + 3, bv[r], bi[r])) { bv[r] = qq.w; bi[r] = b + 3; }
-            }
-          }
+          for (int r = 0; r < GREEDY_ROWS; ++r)
+            if (r < nr) scan_unit(q[1][r], 4 * u2, bv[r], bi[r]);
         }
       }
     } else {
@@ -92,7 +101,7 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
           if (r < nr) q[r] = __ldcs(rows + (size_t)r * V + u);
 #pragma unroll
         for (int r = 0; r < GREEDY_ROWS; ++r)
-          if (r < nr && better(q[r], u, bv[r], bi[r])) { bv[r] = q[r]; bi[r] = u; }
+          if (r < nr && q[r] > bv[r]) { bv[r] = q[r]; bi[r] = u; }
       }
     }
 #pragma unroll
@@ -145,6 +154,8 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
                  const int32_t *__restrict__ draft, const float *__restrict__ u_accept,
                  const float *__restrict__ u_resample, int S, int K, int V,
                  int32_t *__restrict__ accept_len, int32_t *__restrict__ next_token) {
+  pdl_wait();
+  pdl_trigger();
   const int s = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
   __shared__ int s_a;

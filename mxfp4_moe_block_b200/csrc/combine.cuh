@@ -14,6 +14,8 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ pair_row,
                const float *__restrict__ topk_w, int T, int k, int H,
                const uint16_t *residual, uint16_t *out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (t >= T) return;
   const int cbeg = blockIdx.y * blockDim.x * 4;
@@ -52,6 +54,8 @@ combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ pair_row
 // out[t] = bf16( x[t] / sqrt(mean(x[t]^2) + eps) ).  H % 8 == 0.
 __global__ void __launch_bounds__(256)
 rms_norm_kernel(const uint16_t *x, int T, int H, float eps, uint16_t *out) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (t >= T) return;
   const uint16_t *row = x + (size_t)t * H;

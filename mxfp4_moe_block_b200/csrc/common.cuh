@@ -9,6 +9,7 @@
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <stdint.h>
+#include <utility>
 
 #include "../../include/mxfp4_moe.h"
 
@@ -22,6 +23,37 @@ __device__ __forceinline__ void raise_status(int detail) {
 }
 
 constexpr unsigned FULL = 0xffffffffu;
+
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation, so the next kernel on the stream
+// may become resident (and run its prologue) while this one finishes.
+// pdl_wait() blocks until the preceding kernel on the stream has completed
+// and its writes are visible; a kernel calls it before it reads anything a
+// preceding kernel may have written, and before its first global write.
+// pdl_trigger() lets the next kernel launch; kernels call it after their
+// wait, so a kernel that starts early finds everything two launches back
+// complete.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Host: launch `kernel` with programmatic stream serialisation allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // bf16 bit patterns packed two per 32-bit word -> float.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

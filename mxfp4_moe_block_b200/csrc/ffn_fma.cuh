@@ -49,6 +49,8 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
 // x [T, H] bf16 -> float.
 __global__ void __launch_bounds__(256)
 x_to_f32_kernel(const uint16_t *__restrict__ x, size_t n8, float *__restrict__ x32) {
+  pdl_wait();
+  pdl_trigger();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + i);
@@ -169,6 +171,8 @@ __device__ __forceinline__ void ffn1_group(const FfnArgs &a, int e, int n0, int 
 template <int RG>
 __global__ void __launch_bounds__(FMA_THREADS, 1)
 ffn1_fma_kernel(FfnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_act[1024];
   __shared__ int s_n;
   const int n_act = build_active(a.off, a.E, s_act, &s_n);
@@ -213,6 +217,8 @@ __device__ __forceinline__ void ffn2_group(const FfnArgs &a, int e, int m0, int 
 template <int RD>
 __global__ void __launch_bounds__(FMA_THREADS, 1)
 ffn2_fma_kernel(FfnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int s_act[1024];
   __shared__ int s_n;
   const int n_act = build_active(a.off, a.E, s_act, &s_n);

@@ -298,6 +298,8 @@ __device__ __forceinline__ void store_terms_f8(float v, size_t r, int n, int kdi
 __global__ void __launch_bounds__(256)
 split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, int P, int k,
                int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int nb = H / 32;
   const long total = (long)P * nb;
@@ -321,7 +323,13 @@ constexpr int ENC_MAX_PAIRS = 16;
 template <int NT>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp, int k,
-                      int K, uint8_t *__restrict__ q, float *__restrict__ rs) {
+                      int K, uint8_t *__restrict__ q, float *__restrict__ rs, int early_trigger) {
+  // early_trigger: the next kernel (GEMM-2) may start streaming its weights
+  // while this one still waits for GEMM-1; it reads our output only after
+  // its own wait, and nothing of GEMM-1's before it
+  if (early_trigger) pdl_trigger();
+  pdl_wait();
+  if (!early_trigger) pdl_trigger();
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const uint16_t *row = src + (size_t)(sp ? __ldg(sp + r) / k : r) * K;
@@ -531,25 +539,55 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
-        int e, mt, rowB, nB;
+      auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel) {
+        int e, mt, nB;
         decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
-        const int bsel = ncol <= 16 ? 0 : ncol <= 32 ? 1 : ncol <= 64 ? 2 : ncol <= 128 ? 3 : 4;
+        bsel = ncol <= 16 ? 0 : ncol <= 32 ? 1 : ncol <= 64 ? 2 : ncol <= 128 ? 3 : 4;
+        arow = e * a.rows_per_expert + (MODE == 1 ? mt * 64 : mt * 128);
+      };
+      // the box's inner coordinate is in elements (padded E2M1) or bytes
+      // (packed E2M1); both are kt * 128.  Rows 0-63 of the tile, then rows
+      // 64-127 (GEMM-1: gate, then up).
+      auto load_a = [&](int st, int arow, int kt) {
+        uint8_t *sa = smem + st * C::kA;
+        tma_load_2d(sa, &maps.a, kt * 128, arow, &full[st], pol_w);
+        tma_load_2d(sa + 64 * 128, &maps.a, kt * 128, arow + (MODE == 1 ? a.I : 64), &full[st],
+                    pol_w);
+      };
+      auto load_b = [&](int st, int bsel, int rowB, int kt) {
+        tma_load_2d(smem + C::kOffB + st * C::kB, &maps.b[bsel], kt * 128, rowB, &full[st], pol_x);
+      };
+      // Weights depend on no earlier kernel: the first tile's leading stages
+      // of A stream in before the wait for the activation operand.
+      int npre = 0;
+      if ((int)blockIdx.x < n_tiles) {
+        int arow, rowB, bsel;
+        tile_geom(blockIdx.x, arow, rowB, bsel);
+        npre = min(C::kStages, ksteps);
+        for (int kt = 0; kt < npre; ++kt) {
+          mbar_expect_tx(&full[kt], Kd::kABytes + (uint32_t)a.b_box[bsel] * 128u);
+          load_a(kt, arow, kt);
+        }
+        pdl_wait();
+        pdl_trigger();
+        for (int kt = 0; kt < npre; ++kt) load_b(kt, bsel, rowB, kt);
+        issued = npre;
+        stage = npre % C::kStages;
+        phase = npre == C::kStages ? 1u : 0u;
+      } else {
+        pdl_wait();
+        pdl_trigger();
+      }
+      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+        int arow, rowB, bsel;
+        tile_geom(t, arow, rowB, bsel);
         const uint32_t bbytes = (uint32_t)a.b_box[bsel] * 128u;
-        const int arow = e * a.rows_per_expert + (MODE == 1 ? mt * 64 : mt * 128);
-        for (int kt = 0; kt < ksteps; ++kt) {
+        for (int kt = t == (int)blockIdx.x ? npre : 0; kt < ksteps; ++kt) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
-          uint8_t *sa = smem + stage * C::kA;
-          // the box's inner coordinate is in elements (padded E2M1) or bytes
-          // (packed E2M1); both are kt * 128
-          // rows 0-63 of the tile, then rows 64-127 (GEMM-1: gate, then up)
-          tma_load_2d(sa, &maps.a, kt * 128, arow, &full[stage], pol_w);
-          tma_load_2d(sa + 64 * 128, &maps.a, kt * 128, arow + (MODE == 1 ? a.I : 64),
-                      &full[stage], pol_w);
-          tma_load_2d(smem + C::kOffB + stage * C::kB, &maps.b[bsel], kt * 128, rowB,
-                      &full[stage], pol_x);
+          load_a(stage, arow, kt);
+          load_b(stage, bsel, rowB, kt);
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
@@ -569,6 +607,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     // the B rows) go straight into the 32 x 16-byte layout of tcgen05.cp:
     // byte 16*(row%32) + 4*(row/32) + (k-block within the group).
     const uint32_t kb = a.K / 32;            // scale bytes per row
+    if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
     int stage = 0;
     uint32_t phase = 0;
     for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
@@ -679,6 +718,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     // accumulator column T*j + t holds term t of token j of the tile
     const int q = warp - 4;                     // TMEM lane quarter
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    pdl_wait();                                 // row scales in, h / y out
     constexpr int kTokPerLd = 16 / T;           // tokens per 16-column load
     int it = 0;
     for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
@@ -860,12 +900,15 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
                          C::kSmem);
   }
   if (KIND == KIND_F4) {
-    encode_rows_f4_kernel<T><<<(unsigned)P, ENC_THREADS, 0, s>>>(f.x, f.sp, f.k, H, xq,
-                                                                reinterpret_cast<float *>(xs));
+    if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.x, f.sp, f.k, H, xq,
+                   reinterpret_cast<float *>(xs), 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
   } else {
     const long blocks = (long)P * (H / 32);
     const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
-    split_x_kernel<<<grid, 256, 0, s>>>(f.x, f.sp, (int)P, f.k, H, xq, xs);
+    if (launch_pdl(split_x_kernel, grid, 256, 0, s, f.x, f.sp, (int)P, f.k, H, xq, xs) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   TcMaps maps;
   TcArgs a{};
@@ -891,12 +934,14 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.b_rowscale = reinterpret_cast<const float *>(xs);
   a.K = H;
   a.rows_per_expert = 2 * I;
-  tc_gemm_kernel<KIND, 1, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, TC_THREADS, C::kSmem, s, maps, a) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   if (KIND == KIND_F4)
-    encode_rows_f4_kernel<T><<<(unsigned)P, ENC_THREADS, 0, s>>>(f.h, nullptr, 1, I, hq,
-                                                                reinterpret_cast<float *>(hs));
+    if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.h,
+                   (const int32_t *)nullptr, 1, I, hq, reinterpret_cast<float *>(hs), 1) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
   // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
   for (int i = 0; i < 5; ++i)
@@ -908,8 +953,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.b_rowscale = reinterpret_cast<const float *>(hs);
   a.K = I;
   a.rows_per_expert = H;
-  tc_gemm_kernel<KIND, 2, BN><<<sms, TC_THREADS, C::kSmem, s>>>(maps, a);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, TC_THREADS, C::kSmem, s, maps, a) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

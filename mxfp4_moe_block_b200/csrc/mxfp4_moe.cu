@@ -22,6 +22,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
+  bool greedy_attr = false;   // non-portable cluster size allowed for greedy_kernel
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -43,6 +44,17 @@ const DeviceInfo *device_info() {
     d.ready = true;
   }
   return &d;
+}
+
+// Status of a launch made with cudaLaunchKernelEx (the error is returned,
+// and also left in the runtime's last-error slot, which this clears).
+int launched(cudaError_t e) {
+  if (e != cudaSuccess) {
+    fprintf(stderr, "mxfp4_moe: launch failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 
 int launch_status() {
@@ -83,13 +95,13 @@ int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
   if (!logits || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
   const dim3 block(128), grid((unsigned)((T + 3) / 4));
   cudaStream_t s = (cudaStream_t)stream;
-  if (E <= 32) route_topk_kernel<1><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  else if (E <= 64) route_topk_kernel<2><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  else if (E <= 128) route_topk_kernel<4><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  else if (E <= 256) route_topk_kernel<8><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  else if (E <= 512) route_topk_kernel<16><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  else route_topk_kernel<32><<<grid, block, 0, s>>>(logits, T, E, k, topk_idx, topk_w);
-  return launch_status();
+  auto kern = E <= 32    ? route_topk_kernel<1>
+              : E <= 64  ? route_topk_kernel<2>
+              : E <= 128 ? route_topk_kernel<4>
+              : E <= 256 ? route_topk_kernel<8>
+              : E <= 512 ? route_topk_kernel<16>
+                         : route_topk_kernel<32>;
+  return launched(launch_pdl(kern, grid, block, 0, s, logits, T, E, k, topk_idx, topk_w));
 }
 
 // ---------------------------------------------------------------- permute --
@@ -107,9 +119,8 @@ int moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *expert_of
     cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          33 * 1024 * (int)sizeof(int));
   });
-  permute_kernel<<<1, 1024, smem, (cudaStream_t)stream>>>(topk_idx, (int)P, E, expert_offsets,
-                                                           sorted_pair, pair_row);
-  return launch_status();
+  return launched(launch_pdl(permute_kernel, 1, 1024, smem, (cudaStream_t)stream, topk_idx, (int)P,
+                             E, expert_offsets, sorted_pair, pair_row));
 }
 
 // -------------------------------------------------------------------- FFN --
@@ -173,15 +184,13 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
   if (variant == MOE_FFN_TENSOR_F8) return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F8);
   if (variant == MOE_FFN_TENSOR_F4) return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F4);
   const size_t n8 = (size_t)T * H / 8;
-  x_to_f32_kernel<<<(unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8), 256, 0, s>>>(
-      x, n8, a.x32);
-  int st = launch_status();
+  int st = launched(launch_pdl(x_to_f32_kernel,
+                               (unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8),
+                               256, 0, s, x, n8, a.x32));
   if (st != MOE_OK) return st;
-  ffn1_fma_kernel<4><<<dev->sms, FMA_THREADS, 0, s>>>(a);
-  st = launch_status();
+  st = launched(launch_pdl(ffn1_fma_kernel<4>, dev->sms, FMA_THREADS, 0, s, a));
   if (st != MOE_OK) return st;
-  ffn2_fma_kernel<8><<<dev->sms, FMA_THREADS, 0, s>>>(a);
-  return launch_status();
+  return launched(launch_pdl(ffn2_fma_kernel<8>, dev->sms, FMA_THREADS, 0, s, a));
 }
 
 int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
@@ -248,9 +257,8 @@ int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w, in
   if (T == 0) return MOE_OK;
   if (!y || !pair_row || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   const dim3 grid((unsigned)T, (unsigned)((H + 1023) / 1024));
-  combine_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(y, pair_row, topk_w, T, k, H, residual,
-                                                         out);
-  return launch_status();
+  return launched(launch_pdl(combine_kernel, grid, 256, 0, (cudaStream_t)stream, y, pair_row,
+                             topk_w, T, k, H, residual, out));
 }
 
 int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
@@ -258,8 +266,7 @@ int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
   if (T < 0 || H <= 0 || H % 8 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !out) return MOE_ERR_INVALID_ARG;
-  rms_norm_kernel<<<T, 256, 0, (cudaStream_t)stream>>>(x, T, H, eps, out);
-  return launch_status();
+  return launched(launch_pdl(rms_norm_kernel, T, 256, 0, (cudaStream_t)stream, x, T, H, eps, out));
 }
 
 // ----------------------------------------------------------------- accept --
@@ -269,25 +276,36 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
   if (S == 0) return MOE_OK;
   if (!logits || !draft || !accept_len || !next_token) return MOE_ERR_INVALID_ARG;
   if (S > 65535) return MOE_ERR_UNSUPPORTED;
-  const int per_cta = 4 * GREEDY_THREADS;           // elements per CTA and pass
+  DeviceInfo *dev = const_cast<DeviceInfo *>(device_info());
+  if (!dev) return MOE_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (!dev->greedy_attr) {
+      if (cudaFuncSetAttribute(greedy_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+        return launch_status();
+      dev->greedy_attr = true;
+    }
+  }
+  // 1024 threads (128 KB of loads in flight per SM) while the clusters of all
+  // sequences fit on the SMs one CTA each, else 512 (two CTAs per SM)
+  int threads = (long long)S * GREEDY_CLUSTER <= dev->sms ? GREEDY_MAX_THREADS : 512;
   int csize = GREEDY_CLUSTER;
-  while (csize > 1 && (long long)V < (long long)csize * per_cta) csize >>= 1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(greedy_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  });
+  while (csize > 1 && (long long)V < (long long)csize * 4 * threads) csize >>= 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(csize, S, 1);
-  cfg.blockDim = dim3(GREEDY_THREADS, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = (cudaStream_t)stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t err =
       cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, accept_len, next_token);
   if (err != cudaSuccess) {
@@ -308,9 +326,8 @@ int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
   if (S > (1 << 30)) return MOE_ERR_UNSUPPORTED;
   int threads = ((V + 31) / 32) * 32;
   if (threads > 1024) threads = 1024;
-  rejection_kernel<<<S, threads, 0, (cudaStream_t)stream>>>(p, q, draft, u_accept, u_resample,
-                                                            S, K, V, accept_len, next_token);
-  return launch_status();
+  return launched(launch_pdl(rejection_kernel, S, threads, 0, (cudaStream_t)stream, p, q, draft,
+                             u_accept, u_resample, S, K, V, accept_len, next_token));
 }
 
 // ----------------------------------------------------------------- status --

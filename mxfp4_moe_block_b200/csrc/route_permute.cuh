@@ -18,6 +18,8 @@ template <int PER>
 __global__ void __launch_bounds__(128)
 route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
                   int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -69,6 +71,8 @@ __global__ void __launch_bounds__(1024)
 permute_kernel(const int32_t *__restrict__ topk_idx, int P, int E,
                int32_t *__restrict__ expert_offsets,
                int32_t *__restrict__ sorted_pair, int32_t *__restrict__ pair_row) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ int smem[];
   int *cnt = smem;             // [32][E]
   int *offs = smem + 32 * E;   // [E]

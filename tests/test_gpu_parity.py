@@ -235,7 +235,10 @@ def test_greedy_bit_exact(name):
 
 def test_greedy_edges():
     rng = np.random.default_rng(9)
-    for S, K, V in [(3, 1, 1), (5, 32, 1001), (2, 8, 7), (4, 3, 5000)]:
+    # ragged V (scalar path), many ties, one to 32 rows, both CTA sizes
+    # (1024 threads for few sequences, 512 for many), full vocabulary rows
+    for S, K, V in [(3, 1, 1), (5, 32, 1001), (2, 8, 7), (4, 3, 5000), (1, 8, 152064),
+                    (20, 5, 70000), (300, 2, 4096), (1, 16, 152063)]:
         lg = rng.integers(-3, 3, (S, K, V)).astype(np.float32)       # many ties
         am = lg.argmax(-1).astype(np.int32)
         for d in (am, np.where(rng.random((S, K)) < 0.3, (am + 1) % V, am).astype(np.int32)):

@@ -89,6 +89,12 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
   }
 }
 
+// Inline first try; the bounded slow path only when the phase is not done.
+__device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity,
+                                               volatile int *abort) {
+  return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort);
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
                                             uint64_t *bar, uint64_t policy) {
   asm volatile(
@@ -584,7 +590,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         tile_geom(t, arow, rowB, bsel);
         const uint32_t bbytes = (uint32_t)a.b_box[bsel] * 128u;
         for (int kt = t == (int)blockIdx.x ? npre : 0; kt < ksteps; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+          if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
           load_a(stage, arow, kt);
           load_b(stage, bsel, rowB, kt);
@@ -614,21 +620,25 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       int e, mt, rowB, nB;
       decode(t, e, mt, rowB, nB);
       const int ebase = e * a.rows_per_expert;
+      // this lane's four A rows (lane + 32q) for the whole tile
+      const uint8_t *src_a[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = lane + 32 * q;
+        const int row = MODE == 1 ? ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64)
+                                  : ebase + mt * 128 + i;
+        src_a[q] = a.a_scales + (size_t)row * kb;
+      }
       for (int kt = 0; kt < ksteps; ++kt) {
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+        if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
         uint8_t *sfa = smem + C::kOffSfa + stage * C::kSfa;
         uint8_t *sfb = smem + C::kOffSfb + stage * C::kSfb;
 #pragma unroll
         for (int g = 0; g < Kd::kKGroups; ++g) {
           const uint32_t koff = (uint32_t)(kt * Kd::kKGroups + g) * 4;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {       // A rows lane + 32q
-            const int i = lane + 32 * q;
-            int row;
-            if (MODE == 1) row = ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64);
-            else row = ebase + mt * 128 + i;
-            cp_async4(sfa + 512 * g + 16 * lane + 4 * q, a.a_scales + (size_t)row * kb + koff);
-          }
+          for (int q = 0; q < 4; ++q)         // A rows lane + 32q
+            cp_async4(sfa + 512 * g + 16 * lane + 4 * q, src_a[q] + koff);
 #pragma unroll
           for (int q = 0; q < 4 * C::kRowChunks; ++q) {
             const int i = lane + 32 * q;
@@ -656,19 +666,32 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                         smem_desc(smem_u32(smem + C::kOffSfbConst + 512 * c), 0, 128,
                                   kSwizzleNone));
       }
+      // Descriptors of stage 0.  A stage's operands, and each MMA's K slice,
+      // sit at fixed byte offsets from these, and the start-address field
+      // (address >> 4, 14 bits; shared memory is below 256 KB) takes such an
+      // offset by plain addition -- the single issuing thread does little
+      // more per MMA than the instruction itself.
+      const uint64_t a_desc0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
+      const uint64_t b_desc0 = smem_desc(smem_u32(smem + C::kOffB), 16, 1024, kSwizzle128B);
+      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + C::kOffSfa), 0, 128, kSwizzleNone);
+      const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + C::kOffSfb), 0, 128, kSwizzleNone);
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
         int e, mt, rowB, nB;
         decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
+        // the tile's instruction descriptor; MMA kk or-s in its scale byte
+        // selector (sf_id, bits 4-5 and 29-30)
+        const uint32_t idesc0 =
+            KIND == KIND_F4 ? idesc_block_scaled(1, 1, ncol, 0) : idesc_block_scaled(5, 0, ncol, 0);
         const int buf = it % C::kAcc;
         const uint32_t use = (uint32_t)(it / C::kAcc);
-        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort)) break;
+        if (!mbar_wait_fast(&acc_empty[buf], (use & 1) ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
         bool ok = true;
         for (int kt = 0; kt < ksteps; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort)) { ok = false; break; }
+          if (!mbar_wait_fast(&full[stage], phase, abort)) { ok = false; break; }
           // The scale bytes arrive by cp.async and are tracked by the same
           // mbarrier; as in CUTLASS's cp.async-fed UMMA pipelines, the barrier
           // wait is the only ordering tcgen05.cp needs.
@@ -676,34 +699,36 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           // TMEM: per stage, the A scale groups then, per group, the B row chunks
           const uint32_t sfa_t = tmem + sf_col0 + stage * C::kSfCols;
           const uint32_t sfb_t = sfa_t + 4 * Kd::kKGroups;
-          const uint32_t sa = smem_u32(smem + C::kOffSfa + stage * C::kSfa);
-          const uint32_t sb = smem_u32(smem + C::kOffSfb + stage * C::kSfb);
+          const uint64_t sfa_d = sfa_desc0 + (uint64_t)((stage * C::kSfa) >> 4);
+          const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * C::kSfb) >> 4);
 #pragma unroll
           for (int g = 0; g < Kd::kKGroups; ++g) {
-            tc_cp_32x128b(sfa_t + 4 * g, smem_desc(sa + 512 * g, 0, 128, kSwizzleNone));
+            tc_cp_32x128b(sfa_t + 4 * g, sfa_d + (uint64_t)(32 * g));       // 512 B apart
             if (!Kd::kRowScaledB)
 #pragma unroll
             for (int c = 0; c < C::kRowChunks; ++c)
               tc_cp_32x128b(sfb_t + 4 * (g * C::kRowChunks + c),
-                            smem_desc(sb + 512 * (g * C::kRowChunks + c), 0, 128, kSwizzleNone));
+                            sfb_d + (uint64_t)(32 * (g * C::kRowChunks + c)));
           }
-          const uint32_t a_addr = smem_u32(smem + stage * C::kA);
-          const uint32_t b_addr = smem_u32(smem + C::kOffB + stage * C::kB);
+          const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kA) >> 4);
+          const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kB) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            // 32 bytes of each 128-byte row per MMA (K = 32 E4M3/E2M1-padded or 64 E2M1)
-            const uint64_t ad = smem_desc(a_addr + 32 * kk, 16, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(b_addr + 32 * kk, 16, 1024, kSwizzle128B);
+            // 32 bytes of each 128-byte row per MMA (K = 32 E4M3/E2M1-padded or
+            // 64 E2M1): descriptor offset 2 (units of 16 bytes)
             const uint32_t acc = (kt > 0 || kk >= C::kChains) ? 1u : 0u;
             const uint32_t d_t = acc_t + (uint32_t)((kk % C::kChains) * BN);
             if (KIND == KIND_F4) {
               const int g = kk >> 1;                     // scale group of this MMA
               const uint32_t sfid = 2u * (kk & 1);      // two scale bytes per row
-              mma_mxf4(d_t, ad, bd, idesc_block_scaled(1, 1, ncol, sfid),
-                       (sfa_t + 4 * g) | (sfid << 30), sfb_const_t | (sfid << 30), acc);
+              mma_mxf4(d_t, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                       idesc0 | (sfid << 4) | (sfid << 29), (sfa_t + 4 * g) | (sfid << 30),
+                       sfb_const_t | (sfid << 30), acc);
             } else {
-              mma_mxf8f6f4(d_t, ad, bd, idesc_block_scaled(5, 0, ncol, kk),
-                           sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30), acc);
+              const uint32_t sfid = (uint32_t)kk;
+              mma_mxf8f6f4(d_t, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                           idesc0 | (sfid << 4) | (sfid << 29), sfa_t | (sfid << 30),
+                           sfb_t | (sfid << 30), acc);
             }
           }
           tc_commit(&empty[stage]);
@@ -726,7 +751,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       decode(t, e, mt, rowB, nB);
       const int buf = it % C::kAcc;
       const uint32_t use = (uint32_t)(it / C::kAcc);
-      if (!mbar_wait(&acc_full[buf], use & 1, abort)) break;
+      if (!mbar_wait_fast(&acc_full[buf], use & 1, abort)) break;
       tc_fence_after();
       const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
       const int ntok = nB / T;                  // tokens in this tile

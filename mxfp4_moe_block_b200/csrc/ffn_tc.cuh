@@ -200,6 +200,21 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x N columns of 32-bit words from registers (this warp's lane quarter).
+__device__ __forceinline__ void tc_st_x4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tc_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                   taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
@@ -440,7 +455,9 @@ struct TcCfg {
                 "descriptor alignment");
 };
 
-constexpr int TC_THREADS = 256;
+// warps: 0 TMA producer, 1 scale loader, 2 TMEM + MMA issuer, 3 constant B
+// scales, 4-7 epilogue, 8-11 A-scale writers (one per TMEM lane quarter)
+constexpr int TC_THREADS = 384;
 
 template <int KIND, int MODE, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -456,6 +473,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   uint64_t *acc_empty = acc_full + 2;          // [2]
   volatile int *abort = reinterpret_cast<volatile int *>(acc_empty + 2);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 3);
+  uint64_t *sfs_full = acc_empty + 4;          // [kStages] scale bytes landed in smem
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
   int *s_act = reinterpret_cast<int *>(smem + C::kOffTab);
   int *s_pre = s_act + 1025;       // tile prefix over active experts
@@ -492,8 +510,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1 + 32);     // producer expect_tx + 32 scale-loader lanes
+      mbar_init(&full[s], 1 + 4);      // producer expect_tx + 4 A-scale writer warps
       mbar_init(&empty[s], 1);         // MMA commit
+      mbar_init(&sfs_full[s], 32);     // 32 scale-loader lanes (cp.async)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -647,7 +666,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                         a.b_scales + (size_t)(rowB + i) * kb + koff);
           }
         }
-        cp_async_arrive_noinc(&full[stage]);
+        cp_async_arrive_noinc(&sfs_full[stage]);
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -673,7 +692,6 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       // more per MMA than the instruction itself.
       const uint64_t a_desc0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
       const uint64_t b_desc0 = smem_desc(smem_u32(smem + C::kOffB), 16, 1024, kSwizzle128B);
-      const uint64_t sfa_desc0 = smem_desc(smem_u32(smem + C::kOffSfa), 0, 128, kSwizzleNone);
       const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + C::kOffSfb), 0, 128, kSwizzleNone);
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
@@ -692,18 +710,19 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         bool ok = true;
         for (int kt = 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&full[stage], phase, abort)) { ok = false; break; }
-          // The scale bytes arrive by cp.async and are tracked by the same
-          // mbarrier; as in CUTLASS's cp.async-fed UMMA pipelines, the barrier
+          // The full barrier completes once the stage's TMA bytes have landed
+          // and the writer warps have stored its A scales into tensor memory
+          // (tcgen05.wait::st + fence before their arrive).  kind::mxf8f6f4's B
+          // block scales reached shared memory by cp.async before the writers
+          // saw them; as in CUTLASS's cp.async-fed UMMA pipelines, the barrier
           // wait is the only ordering tcgen05.cp needs.
           tc_fence_after();
           // TMEM: per stage, the A scale groups then, per group, the B row chunks
           const uint32_t sfa_t = tmem + sf_col0 + stage * C::kSfCols;
           const uint32_t sfb_t = sfa_t + 4 * Kd::kKGroups;
-          const uint64_t sfa_d = sfa_desc0 + (uint64_t)((stage * C::kSfa) >> 4);
           const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * C::kSfb) >> 4);
 #pragma unroll
           for (int g = 0; g < Kd::kKGroups; ++g) {
-            tc_cp_32x128b(sfa_t + 4 * g, sfa_d + (uint64_t)(32 * g));       // 512 B apart
             if (!Kd::kRowScaledB)
 #pragma unroll
             for (int c = 0; c < C::kRowChunks; ++c)
@@ -736,6 +755,43 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         }
         if (!ok) break;
         tc_commit(&acc_full[buf]);
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------- A-scale writers --
+    // Warp 8+q stores lane quarter q of every stage's A scale columns with
+    // tcgen05.st (the scale-factor layout repeats the same 32 lanes in all
+    // four quarters), keeping the copies off the MMA issue path.  Column
+    // 4g + j, lane l = the 4 scale bytes of tile row 32j + l, K-group g: the
+    // 16 bytes the scale loader put at 512g + 16l.
+    const int q = warp - 8;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+      for (int kt = 0; kt < ksteps; ++kt) {
+        // the MMAs that read this stage's columns last time are done, and the
+        // stage's scale bytes are in shared memory
+        if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
+        if (!mbar_wait_fast(&sfs_full[stage], phase, abort)) break;
+        tc_fence_after();
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(smem + C::kOffSfa + stage * C::kSfa) + lane;
+        const uint32_t dst = tmem + lane_base + (uint32_t)C::kAccCols + stage * C::kSfCols;
+        if (Kd::kKGroups == 2) {
+          const uint4 g0 = src[0], g1 = src[32];
+          const uint32_t r[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+          tc_st_x8(dst, r);
+        } else {
+          const uint4 g0 = src[0];
+          const uint32_t r[4] = {g0.x, g0.y, g0.z, g0.w};
+          tc_st_x4(dst, r);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
     }
   } else if (warp >= 4) {

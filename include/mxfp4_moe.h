@@ -216,8 +216,14 @@ int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
  *   draft[s,i] for all i < a (argmax ties to the lowest token id);
  *   next_token = argmax(logits[s, a]) if a < K, else -1.
  *   logits [S, K, V] float, draft [S, K] int32,
- *   accept_len [S] int32 out, next_token [S] int32 out.
- *   Limits: 1 <= K <= 32, 1 <= V < 2^31.
+ *   accept_len [S] int32 out, next_token [S] int32 out.  Until the call
+ *   completes on the stream, the two outputs also hold its per-sequence
+ *   working state (the smallest mismatch key and the rows reported); no
+ *   other memory is used.  Two kernels run: a one-CTA setup, then one
+ *   thread-block cluster per block row.
+ *   Limits: 1 <= K <= 32, 1 <= V <= 2^26, S <= 65535 (else
+ *   MOE_ERR_UNSUPPORTED).  A draft token outside [0, V) sets the device
+ *   status MOE_DEV_BAD_TOKEN and counts as a mismatch.
  */
 int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
                         int V, int32_t *accept_len, int32_t *next_token,

@@ -2,10 +2,14 @@
 //
 // Greedy: the target keeps the confirmed draft tokens and takes over at the
 // first wrong one ("如何评价小米6月9日发布的MiMo-V2.5-Pro-UltraSpeed模式？",
-// section "二、投机解码").  One thread-block cluster per sequence: CTA r of the
-// cluster scans slice r of every row of the block (coalesced 16-byte loads),
-// the per-row partial argmaxes meet in CTA 0 through distributed shared
-// memory, and CTA 0 finds the first mismatch with a warp ballot.
+// section "二、投机解码").  One thread-block cluster per block row (s, i):
+// CTA r of the cluster scans slice r of the row with coalesced 16-byte
+// loads, the partial argmaxes meet in CTA 0 through distributed shared
+// memory, and CTA 0 reports a mismatching row as the 32-bit key
+// (i << 26 | argmax) to an atomicMin on the sequence's slot; the last of the
+// K rows to report turns the minimum into (accept_len, next_token).  The
+// slots are accept_len / next_token themselves, set up by a one-CTA kernel
+// launched just before.
 //
 // Rejection sampling ("MiMo-v2.5-Pro-UltraSpeed - infra 架构解读", section
 // "数据流概览"): exact test u*q(x) < p(x) in double, first rejection by
@@ -19,9 +23,11 @@
 namespace moe {
 namespace cg = cooperative_groups;
 
-constexpr int GREEDY_MAX_THREADS = 1024;
-constexpr int GREEDY_ROWS = 4;       // rows scanned together
-constexpr int GREEDY_CLUSTER = 16;   // CTAs per sequence (non-portable cluster size)
+constexpr int GREEDY_THREADS = 256;
+constexpr int GREEDY_UNROLL = 8;         // 16-byte loads in flight per thread
+constexpr int GREEDY_MAX_CLUSTER = 16;   // CTAs per row (non-portable cluster size)
+constexpr int GREEDY_TOKEN_BITS = 26;    // key = row << 26 | token; V <= 2^26
+constexpr unsigned GREEDY_NO_MISS = 0xffffffffu;
 
 // One 16-byte unit of a row (elements b..b+3), visited in increasing index
 // order by this thread: the running (bv, bi) keeps the first occurrence of
@@ -35,114 +41,102 @@ __device__ __forceinline__ void scan_unit(const float4 q, int b, float &bv, int 
   }
 }
 
-// grid (cluster_size, S), cluster (cluster_size, 1, 1), blockDim a multiple
-// of 32 up to 1024.  CTA r of a sequence's cluster owns slice r of [0, V) of
-// every row; a thread walks its units of that slice for up to 8 rows at once
-// in increasing index order, keeping one (value, index) candidate per row;
-// warps, then the CTA, then the cluster (through distributed shared memory)
-// reduce the candidates with the lowest-index tie rule.  Rows hold finite
-// values (a row of -inf has no candidate and never matches a draft).
-__global__ void __launch_bounds__(GREEDY_MAX_THREADS, 1)
+// Per sequence: accept_len[s] becomes the minimum-key slot (no mismatch
+// yet), next_token[s] the count of rows reported.
+__global__ void __launch_bounds__(256)
+greedy_init_kernel(int S, int32_t *__restrict__ accept_len, int32_t *__restrict__ next_token) {
+  pdl_wait();
+  pdl_trigger();
+  for (int s = blockIdx.x * blockDim.x + threadIdx.x; s < S; s += gridDim.x * blockDim.x) {
+    accept_len[s] = (int32_t)GREEDY_NO_MISS;
+    next_token[s] = 0;
+  }
+}
+
+// grid (cluster_size, K, S), cluster (cluster_size, 1, 1), GREEDY_THREADS.
+// Rows hold finite values (a row of -inf reports token 0).
+__global__ void __launch_bounds__(GREEDY_THREADS)
 greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draft,
               int S, int K, int V, int32_t *__restrict__ accept_len,
               int32_t *__restrict__ next_token) {
-  pdl_wait();
-  pdl_trigger();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int ncta = (int)cluster.num_blocks();
-  const int s = blockIdx.y;
+  const int i = blockIdx.y, s = blockIdx.z;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  __shared__ float part_v[32];
-  __shared__ int part_i[32];
-  __shared__ float red_v[GREEDY_MAX_THREADS / 32][32];
-  __shared__ int red_i[GREEDY_MAX_THREADS / 32][32];
+  const int bd = blockDim.x;
+  __shared__ float red_v[GREEDY_THREADS / 32];
+  __shared__ int red_i[GREEDY_THREADS / 32];
+  __shared__ float part_v;
+  __shared__ int part_i;
 
-  const bool vec = (V & 3) == 0;       // rows 16-byte aligned: float4 units
-  const int units = vec ? V / 4 : V;
-  const int per = (units + ncta - 1) / ncta;
-  const int u0 = min(units, rank * per), u1 = min(units, u0 + per);
-
-  for (int i0 = 0; i0 < K; i0 += GREEDY_ROWS) {
-    const int nr = min(GREEDY_ROWS, K - i0);
-    const float *rows = logits + ((size_t)s * K + i0) * V;
-    float bv[GREEDY_ROWS];
-    int bi[GREEDY_ROWS];
+  // The logits were complete before the setup kernel passed its own wait,
+  // so the scan needs no wait; only the slots do.
+  const float *row = logits + ((size_t)s * K + i) * V;
+  float bv = -INFINITY;
+  int bi = -1;
+  if ((V & 3) == 0) {                  // rows 16-byte aligned: float4 units
+    const int units = V / 4;
+    const int per = (units + ncta - 1) / ncta;
+    const int u0 = min(units, rank * per), u1 = min(units, u0 + per);
+    const float4 *row4 = reinterpret_cast<const float4 *>(row);
+    for (int u = u0 + threadIdx.x; u < u1; u += GREEDY_UNROLL * bd) {
+      float4 q[GREEDY_UNROLL];
 #pragma unroll
-    for (int r = 0; r < GREEDY_ROWS; ++r) { bv[r] = -INFINITY; bi[r] = -1; }
-    if (vec) {
-      // two strided units per iteration: 2 x GREEDY_ROWS independent
-      // 16-byte loads in flight per thread, consumed in index order
-      const float4 *rows4 = reinterpret_cast<const float4 *>(rows);
-      const int step = blockDim.x;
-      for (int u = u0 + threadIdx.x; u < u1; u += 2 * step) {
-        const int u2 = u + step;
-        float4 q[2][GREEDY_ROWS];
+      for (int j = 0; j < GREEDY_UNROLL; ++j)
+        if (u + j * bd < u1) q[j] = __ldcs(row4 + u + j * bd);
 #pragma unroll
-        for (int r = 0; r < GREEDY_ROWS; ++r) {
-          const float4 *p = rows4 + (size_t)r * units;
-          if (r < nr) q[0][r] = __ldcs(p + u);
-          if (r < nr && u2 < u1) q[1][r] = __ldcs(p + u2);
-        }
-#pragma unroll
-        for (int r = 0; r < GREEDY_ROWS; ++r)
-          if (r < nr) scan_unit(q[0][r], 4 * u, bv[r], bi[r]);
-        if (u2 < u1) {
-#pragma unroll
-          for (int r = 0; r < GREEDY_ROWS; ++r)
-            if (r < nr) scan_unit(q[1][r], 4 * u2, bv[r], bi[r]);
-        }
-      }
-    } else {
-      for (int u = u0 + threadIdx.x; u < u1; u += blockDim.x) {
-        float q[GREEDY_ROWS];
-#pragma unroll
-        for (int r = 0; r < GREEDY_ROWS; ++r)
-          if (r < nr) q[r] = __ldcs(rows + (size_t)r * V + u);
-#pragma unroll
-        for (int r = 0; r < GREEDY_ROWS; ++r)
-          if (r < nr && q[r] > bv[r]) { bv[r] = q[r]; bi[r] = u; }
-      }
+      for (int j = 0; j < GREEDY_UNROLL; ++j)
+        if (u + j * bd < u1) scan_unit(q[j], 4 * (u + j * bd), bv, bi);
     }
+  } else {
+    const int per = (V + ncta - 1) / ncta;
+    const int v0 = min(V, rank * per), v1 = min(V, v0 + per);
+    for (int v = v0 + threadIdx.x; v < v1; v += GREEDY_UNROLL * bd) {
+      float q[GREEDY_UNROLL];
 #pragma unroll
-    for (int r = 0; r < GREEDY_ROWS; ++r) {
-      warp_argmax(bv[r], bi[r]);
-      if (lane == 0 && r < nr) { red_v[w][i0 + r] = bv[r]; red_i[w][i0 + r] = bi[r]; }
+      for (int j = 0; j < GREEDY_UNROLL; ++j)
+        if (v + j * bd < v1) q[j] = __ldcs(row + v + j * bd);
+#pragma unroll
+      for (int j = 0; j < GREEDY_UNROLL; ++j)
+        if (v + j * bd < v1 && q[j] > bv) { bv = q[j]; bi = v + j * bd; }
     }
   }
+  warp_argmax(bv, bi);
+  if (lane == 0) { red_v[w] = bv; red_i[w] = bi; }
   __syncthreads();
-  if (threadIdx.x < K) {
-    const int i = threadIdx.x;
-    float v = 0.f;
+  if (threadIdx.x == 0) {
+    float v = -INFINITY;
     int idx = -1;
     for (int ww = 0; ww < nw; ++ww)
-      if (better(red_v[ww][i], red_i[ww][i], v, idx)) { v = red_v[ww][i]; idx = red_i[ww][i]; }
-    part_v[i] = v;
-    part_i[i] = idx;
+      if (better(red_v[ww], red_i[ww], v, idx)) { v = red_v[ww]; idx = red_i[ww]; }
+    part_v = v;
+    part_i = idx;
   }
   cluster.sync();
-  if (rank == 0 && threadIdx.x < 32) {
-    const int i = threadIdx.x;
-    float bv = 0.f;
-    int bi = -1;
-    if (i < K) {
-      for (int r = 0; r < ncta; ++r) {
-        const float *pv = cluster.map_shared_rank(part_v, r);
-        const int *pi = cluster.map_shared_rank(part_i, r);
-        if (better(pv[i], pi[i], bv, bi)) { bv = pv[i]; bi = pi[i]; }
-      }
+  if (rank == 0 && threadIdx.x == 0) {
+    float v = -INFINITY;
+    int m = -1;
+    for (int r = 0; r < ncta; ++r) {
+      const float pv = *cluster.map_shared_rank(&part_v, r);
+      const int pi = *cluster.map_shared_rank(&part_i, r);
+      if (better(pv, pi, v, m)) { v = pv; m = pi; }
     }
-    int d = -1;
-    if (i < K) {
-      d = __ldg(draft + (size_t)s * K + i);
-      if (d < 0 || d >= V) raise_status(MOE_DEV_BAD_TOKEN);
-    }
-    const unsigned miss = __ballot_sync(FULL, i < K && d != bi);
-    const int a = miss ? __ffs(miss) - 1 : K;
-    const int nt = __shfl_sync(FULL, bi, a < K ? a : 0);
-    if (i == 0) {
-      accept_len[s] = a;
-      next_token[s] = a < K ? nt : -1;
+    m = max(m, 0);
+    const int d = __ldg(draft + (size_t)s * K + i);
+    if (d < 0 || d >= V) raise_status(MOE_DEV_BAD_TOKEN);
+    pdl_wait();                      // the slots were set up by greedy_init_kernel
+    pdl_trigger();
+    unsigned *key = reinterpret_cast<unsigned *>(accept_len + s);
+    unsigned *cnt = reinterpret_cast<unsigned *>(next_token + s);
+    if (d != m) atomicMin(key, ((unsigned)i << GREEDY_TOKEN_BITS) | (unsigned)m);
+    __threadfence();
+    if (atomicAdd(cnt, 1u) == (unsigned)(K - 1)) {      // the last row of the sequence
+      __threadfence();
+      const unsigned k = atomicOr(key, 0u);
+      const bool miss = k != GREEDY_NO_MISS;
+      accept_len[s] = miss ? (int32_t)(k >> GREEDY_TOKEN_BITS) : K;
+      next_token[s] = miss ? (int32_t)(k & ((1u << GREEDY_TOKEN_BITS) - 1)) : -1;
     }
   }
   cluster.sync();   // keep every CTA's shared memory alive until CTA 0 is done

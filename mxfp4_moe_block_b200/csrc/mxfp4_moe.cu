@@ -275,7 +275,7 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
   if (S < 0 || K < 1 || K > 32 || V < 1) return MOE_ERR_INVALID_ARG;
   if (S == 0) return MOE_OK;
   if (!logits || !draft || !accept_len || !next_token) return MOE_ERR_INVALID_ARG;
-  if (S > 65535) return MOE_ERR_UNSUPPORTED;
+  if (S > 65535 || V > (1 << GREEDY_TOKEN_BITS)) return MOE_ERR_UNSUPPORTED;
   DeviceInfo *dev = const_cast<DeviceInfo *>(device_info());
   if (!dev) return MOE_ERR_CUDA;
   {
@@ -287,33 +287,34 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
       dev->greedy_attr = true;
     }
   }
-  // 1024 threads (128 KB of loads in flight per SM) while the clusters of all
-  // sequences fit on the SMs one CTA each, else 512 (two CTAs per SM)
-  int threads = (long long)S * GREEDY_CLUSTER <= dev->sms ? GREEDY_MAX_THREADS : 512;
-  int csize = GREEDY_CLUSTER;
-  while (csize > 1 && (long long)V < (long long)csize * 4 * threads) csize >>= 1;
+  const cudaStream_t s = (cudaStream_t)stream;
+  // Cluster size per row: slices of about 48 KB, at least two CTAs per SM
+  // over all rows, at least GREEDY_THREADS elements (or float4 units) each.
+  const long long rows = (long long)S * K;
+  const long long units = (V & 3) == 0 ? V / 4 : V;
+  long long csize = std::max<long long>((4LL * V + 49151) / 49152, (2LL * dev->sms + rows - 1) / rows);
+  csize = std::min<long long>(csize, std::max<long long>(1, units / GREEDY_THREADS));
+  csize = std::max<long long>(1, std::min<long long>(csize, GREEDY_MAX_CLUSTER));
+
+  int st = launched(launch_pdl(greedy_init_kernel, (unsigned)std::min<long long>((S + 255) / 256, 256),
+                               256, 0, s, S, accept_len, next_token));
+  if (st != MOE_OK) return st;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(csize, S, 1);
-  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.gridDim = dim3((unsigned)csize, (unsigned)K, (unsigned)S);
+  cfg.blockDim = dim3(GREEDY_THREADS, 1, 1);
   cfg.dynamicSmemBytes = 0;
-  cfg.stream = (cudaStream_t)stream;
+  cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.x = (unsigned)csize;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t err =
-      cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, accept_len, next_token);
-  if (err != cudaSuccess) {
-    fprintf(stderr, "mxfp4_moe: cluster launch failed: %s\n", cudaGetErrorString(err));
-    cudaGetLastError();
-    return MOE_ERR_CUDA;
-  }
-  return launch_status();
+  return launched(
+      cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, accept_len, next_token));
 }
 
 int block_accept_rejection(const float *p, const float *q, const int32_t *draft,

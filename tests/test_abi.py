@@ -51,3 +51,6 @@ def test_host_only_calls(library):
     # argument checks return before any CUDA call
     assert library.moe_route_topk(None, 4, 8, 9, None, None, None) == 1
     assert library.block_accept_greedy(None, None, 1, 0, 10, None, None, None) == 1
+    # a vocabulary beyond the greedy key's 26 token bits is refused up front
+    # (non-null dummy addresses: the size check comes before any device use)
+    assert library.block_accept_greedy(16, 16, 1, 8, (1 << 26) + 1, 16, 16, None) == 2

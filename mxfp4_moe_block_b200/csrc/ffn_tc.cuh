@@ -185,7 +185,19 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
       : "memory");
 }
 
-// 32 lanes x 16 columns of 32-bit accumulator -> 16 registers per thread.
+// 32 lanes x 16 columns of 32-bit accumulator -> 16 registers per thread;
+// the registers are valid after tc_wait_ld().
+__device__ __forceinline__ void tc_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(
@@ -417,6 +429,8 @@ struct TcArgs {
   float *y;                  // [P, H]
 };
 
+constexpr int kMaxStages = 12;
+
 template <int KIND, int BN>
 struct TcCfg {
   using Kd = TcKindCfg<KIND>;
@@ -429,7 +443,7 @@ struct TcCfg {
   static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
   static constexpr int kFixed = 1024 + 2048 + 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
   static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
-  static constexpr int kStages = kStages0 > 12 ? 12 : kStages0;
+  static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
   static constexpr int kSfCols =                                    // TMEM columns per stage
       4 * Kd::kKGroups * (Kd::kRowScaledB ? 1 : 1 + kRowChunks);
   static constexpr int kAcc = BN <= 128 ? 2 : 1;                   // accumulator buffers
@@ -807,20 +821,43 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       decode(t, e, mt, rowB, nB);
       const int buf = it % C::kAcc;
       const uint32_t use = (uint32_t)(it / C::kAcc);
+      const int ntok = nB / T;                  // tokens in this tile
+      const int rtok0 = rowB / T;               // sorted row of the tile's first token
+      // the first chunk's row scales do not depend on the accumulator: load
+      // them while the MMAs still run
+      float rs0[16];
+      if (Kd::kRowScaledB) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int tok = min(i / T, ntok - 1);          // rows past ntok are discarded
+          rs0[i] = __ldg(a.b_rowscale + (size_t)(rtok0 + tok) * T + i % T);
+        }
+      }
       if (!mbar_wait_fast(&acc_full[buf], use & 1, abort)) break;
       tc_fence_after();
       const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
-      const int ntok = nB / T;                  // tokens in this tile
-      const int rtok0 = rowB / T;               // sorted row of the tile's first token
       for (int c0 = 0; c0 < nB; c0 += 16) {
         float v[16];
-        tc_ld16(acc_t + lane_base + (uint32_t)c0, v);
+        {
+          uint32_t r[C::kChains][16];
 #pragma unroll
-        for (int ch = 1; ch < C::kChains; ++ch) {
-          float w[16];
-          tc_ld16(acc_t + lane_base + (uint32_t)(ch * BN + c0), w);
+          for (int ch = 0; ch < C::kChains; ++ch)
+            tc_ld16_nowait(acc_t + lane_base + (uint32_t)(ch * BN + c0), r[ch]);
+          tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] += w[i];
+          for (int i = 0; i < 16; ++i) {
+            float acc = __uint_as_float(r[0][i]);
+#pragma unroll
+            for (int ch = 1; ch < C::kChains; ++ch) acc += __uint_as_float(r[ch][i]);
+            v[i] = acc;
+          }
+        }
+        if (c0 + 16 >= nB) {
+          // every accumulator column of the tile is in registers: hand the
+          // buffer back to the MMA warp before the arithmetic and the stores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
         const int tok0 = c0 / T;
         float tok_sum[kTokPerLd];
@@ -828,10 +865,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         for (int j = 0; j < kTokPerLd; ++j) {
           float sum = 0.f;
           if (Kd::kRowScaledB) {
-            const int tok = min(tok0 + j, ntok - 1);     // rows past ntok are discarded
-            const float *rsc = a.b_rowscale + (size_t)(rtok0 + tok) * T;
+            if (c0 == 0) {
 #pragma unroll
-            for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], __ldg(rsc + u), sum);
+              for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], rs0[T * j + u], sum);
+            } else {
+              const int tok = min(tok0 + j, ntok - 1);     // rows past ntok are discarded
+              const float *rsc = a.b_rowscale + (size_t)(rtok0 + tok) * T;
+#pragma unroll
+              for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], __ldg(rsc + u), sum);
+            }
           } else {
 #pragma unroll
             for (int u = 0; u < T; ++u) sum += v[T * j + u];
@@ -869,9 +911,6 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           asm volatile("bar.sync 1, 128;" ::: "memory");
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
 

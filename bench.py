@@ -268,13 +268,34 @@ def e2e_time(wl, variant, steps, warmup):
     for _ in range(warmup):
         one()
     torch.cuda.synchronize()
+    # the whole step -- copies in, the nine kernels, copies out -- as one CUDA
+    # graph (a serving loop replays it; launching it call by call from Python
+    # would measure the interpreter instead)
+    mode = "CUDA graph replay"
+    graph = torch.cuda.CUDAGraph()
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            one()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            one()
+        for _ in range(warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        run = graph.replay
+    except Exception as ex:          # capture refused: time the eager calls
+        mode = f"eager ({type(ex).__name__})"
+        run = one
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for _ in range(steps):
-        one()
+        run()
     b.record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps, h2d, d2h
+    return a.elapsed_time(b) / steps, h2d, d2h, mode
 
 
 # --------------------------------------------------------------- CPU oracle --
@@ -424,9 +445,9 @@ def main():
     ms = max_over_ranks(ms, world, dev)
 
     if args.no_e2e:
-        e2e_ms, h2d, d2h = float("nan"), 0, 0
+        e2e_ms, h2d, d2h, e2e_mode = float("nan"), 0, 0, None
     else:
-        e2e_ms, h2d, d2h = e2e_time(wl, variant, args.steps, 3)
+        e2e_ms, h2d, d2h, e2e_mode = e2e_time(wl, variant, args.steps, 3)
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     peak, peak_kind = load_peaks()
@@ -451,7 +472,7 @@ def main():
                          "eager_step": eager_ms, "graph_step": ms if graph is not None else None},
         "ffn_tflops": wl.ffn_flops() / (ffn_ms * 1e-3) / 1e12,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "timing": e2e_mode},
         "gpu_launches": launches_per_step * args.steps,
         "launches_per_step": launches_per_step,
         "kernels": [n.split("(")[0].split("<")[0].replace("void ", "") for n in kernel_names],

@@ -441,7 +441,7 @@ struct TcCfg {
   static constexpr int kSfb = Kd::kRowScaledB ? 0 : 512 * Kd::kKGroups * kRowChunks;
   static constexpr int kSfbConst = Kd::kRowScaledB ? 512 * kRowChunks : 0;  // all 1.0
   static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
-  static constexpr int kFixed = 1024 + 2048 + 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
+  static constexpr int kFixed = 1024 + 2048 + 1026 * 2 + 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
   static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
   static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
   static constexpr int kSfCols =                                    // TMEM columns per stage
@@ -462,7 +462,9 @@ struct TcCfg {
   static constexpr int kOffBar = kOffSfb + kStages * kSfb;
   static constexpr int kOffXchg = kOffBar + 1024;                // 64 rows x 4 tokens (float)
   static constexpr int kOffTab = kOffXchg + 2048;                 // active list + prefix
-  static constexpr int kOffSfbConst = (kOffTab + 2 * 1025 * 4 + 127) & ~127;  // 16B-aligned for tcgen05.cp
+  // tile table: expert ids (16-bit), tile prefix and first sorted row (32-bit)
+  static constexpr int kTabBytes = 1026 * 2 + 2 * 1025 * 4;
+  static constexpr int kOffSfbConst = (kOffTab + kTabBytes + 127) & ~127;  // 16B-aligned for tcgen05.cp
   static constexpr int kSmem = kOffSfbConst + kSfbConst + 1024;   // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
   static_assert(kOffSfa % 1024 == 0 && kOffSfb % 128 == 0 && kOffSfbConst % 128 == 0,
@@ -489,8 +491,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 3);
   uint64_t *sfs_full = acc_empty + 4;          // [kStages] scale bytes landed in smem
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
-  int *s_act = reinterpret_cast<int *>(smem + C::kOffTab);
-  int *s_pre = s_act + 1025;       // tile prefix over active experts
+  // The table stays small: a GEMM CTA leaves a few KB of the SM's shared
+  // memory free, so that the encode kernels' CTAs can become resident beside
+  // it under programmatic dependent launch.
+  uint16_t *s_act = reinterpret_cast<uint16_t *>(smem + C::kOffTab);   // [1025] (+ count)
+  int *s_pre = reinterpret_cast<int *>(smem + C::kOffTab + 1026 * 2);   // tile prefix
+  int *s_r0 = s_pre + 1025;        // first sorted row of each active expert (+ total)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mtiles = MODE == 1 ? a.I / 64 : a.rows_per_expert / 128;
@@ -501,7 +507,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     int n = 0, acc = 0;
     for (int e0 = 0; e0 < a.E; e0 += 32) {
       const int e = e0 + lane;
-      const int cnt = e < a.E ? __ldg(a.off + e + 1) - __ldg(a.off + e) : 0;
+      const int r0 = e < a.E ? __ldg(a.off + e) : 0;
+      const int cnt = e < a.E ? __ldg(a.off + e + 1) - r0 : 0;
       const int nt = cnt > 0 ? (T * cnt + BN - 1) / BN : 0;
       const unsigned b = __ballot_sync(FULL, nt > 0);
       int sc = nt * mtiles;
@@ -512,15 +519,18 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       }
       if (nt > 0) {
         const int pos = n + __popc(b & lanemask_lt());
-        s_act[pos] = e;
+        s_act[pos] = (uint16_t)e;
         s_pre[pos] = acc + sc - nt * mtiles;   // exclusive
+        s_r0[pos] = r0;
       }
       n += __popc(b);
       acc += __shfl_sync(FULL, sc, 31);
     }
     if (lane == 0) {
-      s_act[1024] = n;
+      s_act[1024] = (uint16_t)n;
       s_pre[n] = acc;
+      s_r0[n] = __ldg(a.off + a.E);   // rows of inactive experts are empty: the next
+                                       // active expert's first row ends the previous one
     }
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -554,15 +564,17 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   const int n_tiles = s_pre[n_act];
 
   // tile index -> (expert, m-block, first B row, B rows in the tile)
+  // Every role walks its tiles in increasing order, so the active-expert
+  // index only moves forward: a linear advance from the last position, all
+  // from shared memory.
+  int dpos = 0;
   auto decode = [&](int t, int &e, int &mt, int &rowB, int &nB) {
-    int lo = 0, hi = n_act - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pre[mid] <= t) lo = mid; else hi = mid - 1;
-    }
+    int lo = dpos;
+    while (lo + 1 < n_act && s_pre[lo + 1] <= t) ++lo;
+    dpos = lo;
     e = s_act[lo];
-    const int r0 = __ldg(a.off + e);
-    const int ne = __ldg(a.off + e + 1) - r0;
+    const int r0 = s_r0[lo];
+    const int ne = s_r0[lo + 1] - r0;
     const int nt_cnt = (T * ne + BN - 1) / BN;
     const int local = t - s_pre[lo];
     mt = local / nt_cnt;

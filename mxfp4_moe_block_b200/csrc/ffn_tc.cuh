@@ -330,9 +330,10 @@ __device__ __forceinline__ void store_terms_f8(float v, size_t r, int n, int kdi
 // bytes.  One warp per 32-element block.
 __global__ void __launch_bounds__(256)
 split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, int P, int k,
-               int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs) {
+               int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs, int *counters) {
   pdl_wait();
   pdl_trigger();
+  if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
   const int lane = threadIdx.x & 31;
   const int nb = H / 32;
   const long total = (long)P * nb;
@@ -356,13 +357,17 @@ constexpr int ENC_MAX_PAIRS = 16;
 template <int NT>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp, int k,
-                      int K, uint8_t *__restrict__ q, float *__restrict__ rs, int early_trigger) {
+                      int K, uint8_t *__restrict__ q, float *__restrict__ rs, int early_trigger,
+                      int *counters) {
   // early_trigger: the next kernel (GEMM-2) may start streaming its weights
   // while this one still waits for GEMM-1; it reads our output only after
   // its own wait, and nothing of GEMM-1's before it
   if (early_trigger) pdl_trigger();
   pdl_wait();
   if (!early_trigger) pdl_trigger();
+  // the GEMMs' tile counters for this call (GEMM-1 reads its own only after
+  // this kernel completed; GEMM-2 after the next one did)
+  if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const uint16_t *row = src + (size_t)(sp ? __ldg(sp + r) / k : r) * K;
@@ -427,6 +432,9 @@ struct TcArgs {
   uint8_t *hs;               // their scale bytes
   // GEMM-2 output
   float *y;                  // [P, H]
+  // tiles past the first wave are handed out by this counter (zeroed by the
+  // encode kernel that runs first in the call)
+  int *tile_counter;
 };
 
 constexpr int kMaxStages = 12;
@@ -474,6 +482,21 @@ struct TcCfg {
 // warps: 0 TMA producer, 1 scale loader, 2 TMEM + MMA issuer, 3 constant B
 // scales, 4-7 epilogue, 8-11 A-scale writers (one per TMEM lane quarter)
 constexpr int TC_THREADS = 384;
+constexpr int kRing = 4;                        // tile indices published ahead
+constexpr int kRingReaders = 1 + 1 + 4 + 4;
+
+// Reader side of the tile ring: tile i of this CTA's sequence (all lanes of
+// the calling warp wait; `arrive` is the one lane that releases the slot).
+__device__ __forceinline__ int ring_read(uint64_t *ring_full, uint64_t *ring_empty,
+                                         volatile int *ring, int i, bool arrive,
+                                         volatile int *abort, int sentinel) {
+  const int slot = i % kRing;
+  if (!mbar_wait_fast(&ring_full[slot], (uint32_t)(i / kRing) & 1u, abort)) return sentinel;
+  const int t = ring[slot];
+  __syncwarp(__activemask());
+  if (arrive) mbar_arrive(&ring_empty[slot]);
+  return t;
+}
 
 template <int KIND, int MODE, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -490,6 +513,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   volatile int *abort = reinterpret_cast<volatile int *>(acc_empty + 2);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 3);
   uint64_t *sfs_full = acc_empty + 4;          // [kStages] scale bytes landed in smem
+  // tile ring: the producer publishes each tile index it takes; every other
+  // role reads the same sequence
+  uint64_t *ring_full = sfs_full + C::kStages;  // [kRing]
+  uint64_t *ring_empty = ring_full + kRing;     // [kRing]
+  volatile int *ring = reinterpret_cast<volatile int *>(ring_empty + kRing);   // [kRing]
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
   // The table stays small: a GEMM CTA leaves a few KB of the SM's shared
   // memory free, so that the encode kernels' CTAs can become resident beside
@@ -537,6 +565,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       mbar_init(&full[s], 1 + 4);      // producer expect_tx + 4 A-scale writer warps
       mbar_init(&empty[s], 1);         // MMA commit
       mbar_init(&sfs_full[s], 32);     // 32 scale-loader lanes (cp.async)
+    }
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&ring_full[r], 1);             // producer
+      mbar_init(&ring_empty[r], kRingReaders); // scale loader, MMA, 4 epilogue, 4 writers
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -609,6 +641,21 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       auto load_b = [&](int st, int bsel, int rowB, int kt) {
         tma_load_2d(smem + C::kOffB + st * C::kB, &maps.b[bsel], kt * 128, rowB, &full[st], pol_x);
       };
+      // Tile sequence: blockIdx.x first, then gridDim.x + (the counter's next
+      // value) -- a CTA whose tiles went fast takes more.  Each index is
+      // published into the ring as soon as it is known.
+      int published = 0;
+      auto publish = [&](int t) {
+        const int slot = published % kRing;
+        if (published >= kRing &&
+            !mbar_wait_fast(&ring_empty[slot], (uint32_t)(published / kRing - 1) & 1u, abort))
+          return false;
+        ring[slot] = t;
+        mbar_arrive(&ring_full[slot]);        // release: the index is visible
+        ++published;
+        return true;
+      };
+      publish(blockIdx.x);
       // Weights depend on no earlier kernel: the first tile's leading stages
       // of A stream in before the wait for the activation operand.
       int npre = 0;
@@ -630,7 +677,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         pdl_wait();
         pdl_trigger();
       }
-      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+      for (int t = blockIdx.x; t < n_tiles && !*abort;) {
+        // the next tile, published before this one's stages are issued
+        const int t_next = (int)gridDim.x + atomicAdd(a.tile_counter, 1);
+        if (!publish(t_next < n_tiles ? t_next : n_tiles)) break;
         int arow, rowB, bsel;
         tile_geom(t, arow, rowB, bsel);
         const uint32_t bbytes = (uint32_t)a.b_box[bsel] * 128u;
@@ -642,7 +692,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
+        t = t_next;
       }
+      if (*abort) publish(n_tiles);            // release readers still waiting
       // drain: wait (bounded) until the last issued stages have landed
       if (*abort) {
         for (int s = 0; s < C::kStages && s < issued; ++s) {
@@ -661,7 +713,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+    int ti = 0;
+    for (int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+         t < n_tiles && !*abort;
+         t = ring_read(ring_full, ring_empty, ring, ++ti, lane == 0, abort, n_tiles)) {
       int e, mt, rowB, nB;
       decode(t, e, mt, rowB, nB);
       const int ebase = e * a.rows_per_expert;
@@ -720,7 +775,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       const uint64_t b_desc0 = smem_desc(smem_u32(smem + C::kOffB), 16, 1024, kSwizzle128B);
       const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + C::kOffSfb), 0, 128, kSwizzleNone);
       int it = 0;
-      for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
+      for (int t = ring_read(ring_full, ring_empty, ring, it, true, abort, n_tiles);
+           t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, true, abort, n_tiles)) {
         int e, mt, rowB, nB;
         decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
@@ -794,7 +850,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+    int ti = 0;
+    for (int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+         t < n_tiles && !*abort;
+         t = ring_read(ring_full, ring_empty, ring, ++ti, lane == 0, abort, n_tiles)) {
       for (int kt = 0; kt < ksteps; ++kt) {
         // the MMAs that read this stage's columns last time are done, and the
         // stage's scale bytes are in shared memory
@@ -828,7 +887,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     pdl_wait();                                 // row scales in, h / y out
     constexpr int kTokPerLd = 16 / T;           // tokens per 16-column load
     int it = 0;
-    for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++it) {
+    for (int t = ring_read(ring_full, ring_empty, ring, it, lane == 0, abort, n_tiles);
+         t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, lane == 0, abort, n_tiles)) {
       int e, mt, rowB, nB;
       decode(t, e, mt, rowB, nB);
       const int buf = it % C::kAcc;
@@ -951,7 +1011,8 @@ inline size_t tc_scale_bytes(size_t P, int K) {
 }
 inline size_t tc_workspace_bytes(size_t P, int H, int I) {
   return align256_tc(tc_term_bytes(P, H)) + align256_tc(tc_scale_bytes(P, H)) +
-         align256_tc(tc_term_bytes(P, I)) + align256_tc(tc_scale_bytes(P, I));
+         align256_tc(tc_term_bytes(P, I)) + align256_tc(tc_scale_bytes(P, I)) +
+         256;                                   // the two GEMMs' tile counters
 }
 
 // The tensor-core variant streams the weights with TMA and needs no
@@ -1020,6 +1081,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   uint8_t *xs = xq + align256_tc(tc_term_bytes(P, H));
   uint8_t *hq = xs + align256_tc(tc_scale_bytes(P, H));
   uint8_t *hs = hq + align256_tc(tc_term_bytes(P, I));
+  int *counters = reinterpret_cast<int *>(hs + align256_tc(tc_scale_bytes(P, I)));
 
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1033,12 +1095,12 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   }
   if (KIND == KIND_F4) {
     if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.x, f.sp, f.k, H, xq,
-                   reinterpret_cast<float *>(xs), 0) != cudaSuccess)
+                   reinterpret_cast<float *>(xs), 0, counters) != cudaSuccess)
       return MOE_ERR_CUDA;
   } else {
     const long blocks = (long)P * (H / 32);
     const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
-    if (launch_pdl(split_x_kernel, grid, 256, 0, s, f.x, f.sp, (int)P, f.k, H, xq, xs) !=
+    if (launch_pdl(split_x_kernel, grid, 256, 0, s, f.x, f.sp, (int)P, f.k, H, xq, xs, counters) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
   }
@@ -1053,6 +1115,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.hq = hq;
   a.hs = hs;
   a.y = f.y;
+  a.tile_counter = counters;
   for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
 
   // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]
@@ -1071,8 +1134,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
 
   if (KIND == KIND_F4)
     if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.h,
-                   (const int32_t *)nullptr, 1, I, hq, reinterpret_cast<float *>(hs), 1) !=
-        cudaSuccess)
+                   (const int32_t *)nullptr, 1, I, hq, reinterpret_cast<float *>(hs), 1,
+                   (int *)nullptr) != cudaSuccess)
       return MOE_ERR_CUDA;
   // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
@@ -1085,6 +1148,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.b_rowscale = reinterpret_cast<const float *>(hs);
   a.K = I;
   a.rows_per_expert = H;
+  a.tile_counter = counters + 1;
   if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, TC_THREADS, C::kSmem, s, maps, a) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;

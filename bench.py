@@ -207,8 +207,7 @@ class Workload:
         mm, s = self.mm, self.sh_r
         if ev is not None:
             ev[0].record()
-        mm.moe_route_topk(self.logits, s.k, self.idx, self.tw)
-        mm.moe_permute(self.idx, s.E, self.off, self.sp, self.pr)
+        mm.moe_route_permute(self.logits, s.k, s.E, self.idx, self.tw, self.off, self.sp, self.pr)
         if ev is not None:
             ev[1].record()
         mm.mxfp4_moe_ffn(self.x, s.k, *self.w, self.off, self.sp, y=self.y, workspace=self.ws,
@@ -243,8 +242,12 @@ def count_launches(wl, variant):
 
 
 def e2e_time(wl, variant, steps, warmup):
-    """Same step through the public API with host buffers: pinned inputs are
-    copied in and the results copied out inside the timed region."""
+    """The same step through the public API with host buffers, as a serving
+    loop runs it: every step's inputs are copied in from pinned host memory
+    and its results (combined hidden states, accept lengths, next tokens)
+    copied out, inside the timed region.  Each step (its kernels and the
+    copies out) is one CUDA graph; the copy in of step i+1 runs on a second
+    stream into the other of two input buffer sets while step i computes."""
     hx = torch.from_numpy(wl.x_bits.view(np.int16)).pin_memory()
     hl = torch.from_numpy(wl.logits_np).pin_memory()
     hb = torch.from_numpy(wl.block_np).pin_memory()
@@ -254,48 +257,72 @@ def e2e_time(wl, variant, steps, warmup):
     hn = torch.empty(wl.nxt.shape, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (hx, hl, hb, hd))
     d2h = sum(t.numel() * t.element_size() for t in (ho, ha, hn))
+    # two input sets on the device: set 0 is the workload's own tensors
+    sets = [(wl.x, wl.logits, wl.block, wl.draft),
+            (torch.empty_like(wl.x), torch.empty_like(wl.logits), torch.empty_like(wl.block),
+             torch.empty_like(wl.draft))]
 
-    def one():
-        wl.x.view(torch.int16).copy_(hx, non_blocking=True)
-        wl.logits.copy_(hl, non_blocking=True)
-        wl.block.copy_(hb, non_blocking=True)
-        wl.draft.copy_(hd, non_blocking=True)
+    def copy_in(i):
+        x, lg, blk, dr = sets[i]
+        x.view(torch.int16).copy_(hx, non_blocking=True)
+        lg.copy_(hl, non_blocking=True)
+        blk.copy_(hb, non_blocking=True)
+        dr.copy_(hd, non_blocking=True)
+
+    def step_out(i):
+        wl.x, wl.logits, wl.block, wl.draft = sets[i]
         wl.step(variant)
         ho.copy_(wl.out, non_blocking=True)
         ha.copy_(wl.acc, non_blocking=True)
         hn.copy_(wl.nxt, non_blocking=True)
 
-    for _ in range(warmup):
-        one()
+    compute = torch.cuda.current_stream()
+    copy = torch.cuda.Stream()
+    for i in (0, 1):
+        copy_in(i)
+        step_out(i)
     torch.cuda.synchronize()
-    # the whole step -- copies in, the nine kernels, copies out -- as one CUDA
-    # graph (a serving loop replays it; launching it call by call from Python
-    # would measure the interpreter instead)
-    mode = "CUDA graph replay"
-    graph = torch.cuda.CUDAGraph()
-    try:
+    graphs = []
+    for i in (0, 1):
         side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
+        side.wait_stream(compute)
         with torch.cuda.stream(side):
-            one()
-        torch.cuda.current_stream().wait_stream(side)
+            step_out(i)
+        compute.wait_stream(side)
         torch.cuda.synchronize()
-        with torch.cuda.graph(graph):
-            one()
-        for _ in range(warmup):
-            graph.replay()
-        torch.cuda.synchronize()
-        run = graph.replay
-    except Exception as ex:          # capture refused: time the eager calls
-        mode = f"eager ({type(ex).__name__})"
-        run = one
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(steps):
-        run()
-    b.record()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step_out(i)
+        graphs.append(g)
+    wl.x, wl.logits, wl.block, wl.draft = sets[0]
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]
+    ev_done = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def run(n):
+        copy.wait_stream(compute)
+        with torch.cuda.stream(copy):
+            copy_in(0)
+            ev_in[0].record(copy)
+        for i in range(n):
+            cur, nxt = i % 2, 1 - i % 2
+            if i + 1 < n:
+                if i >= 1:
+                    copy.wait_event(ev_done[nxt])     # step i-1 has read set nxt
+                with torch.cuda.stream(copy):
+                    copy_in(nxt)
+                    ev_in[nxt].record(copy)
+            compute.wait_event(ev_in[cur])
+            graphs[cur].replay()
+            ev_done[cur].record(compute)
+
+    run(warmup)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps, h2d, d2h, mode
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(compute)
+    run(steps)
+    b.record(compute)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps, h2d, d2h, "CUDA graph per step, copy-in of the next step overlapped"
 
 
 # --------------------------------------------------------------- CPU oracle --

@@ -99,6 +99,18 @@ int moe_permute(const int32_t *topk_idx, int T, int k, int E,
                 int32_t *pair_row, moe_stream_t stream);
 
 /*
+ * moe_route_permute -- moe_route_topk followed by moe_permute, same
+ *   arguments, outputs and errors as the two calls.  For T <= 128 tokens it
+ *   runs as one kernel (one CTA routes every token, then groups the pairs),
+ *   saving a launch on the verify step's critical path; larger batches make
+ *   the two launches.  The pages describe routing and grouping as separate
+ *   steps; fusing them changes no result.
+ */
+int moe_route_permute(const float *logits, int T, int E, int k, int32_t *topk_idx,
+                      float *topk_w, int32_t *expert_offsets, int32_t *sorted_pair,
+                      int32_t *pair_row, moe_stream_t stream);
+
+/*
  * mxfp4_moe_ffn -- SwiGLU FFN of every permuted pair over MXFP4 experts.
  *   The experts hold OCP MXFP4 weights while the rest of the model keeps
  *   higher precision ([P1] "接受率预测与动态回退机制"; [P3] "FP4 Expert 量化";

@@ -28,6 +28,7 @@ SIGNATURES = {
     "moe_version": (_c_int, []),
     "moe_route_topk": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "moe_permute": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp]),
+    "moe_route_permute": (_c_int, [_vp, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "mxfp4_moe_ffn_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
     "mxfp4_moe_ffn": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_size, _vp]),
@@ -120,6 +121,27 @@ def moe_permute(topk_idx, E, expert_offsets=None, sorted_pair=None, pair_row=Non
                              _ptr(expert_offsets, torch.int32), _ptr(sorted_pair, torch.int32),
                              _ptr(pair_row, torch.int32), _stream(stream)), "moe_permute")
     return expert_offsets, sorted_pair, pair_row
+
+
+def moe_route_permute(logits, k, E=None, topk_idx=None, topk_w=None, expert_offsets=None,
+                      sorted_pair=None, pair_row=None, stream=None):
+    """moe_route_topk + moe_permute in one call (one kernel for T <= 128)."""
+    T, E_ = logits.shape
+    E = E_ if E is None else E
+    dev = logits.device
+    P = T * k
+    i32 = dict(dtype=torch.int32, device=dev)
+    topk_idx = torch.empty((T, k), **i32) if topk_idx is None else topk_idx
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_w is None else topk_w
+    expert_offsets = torch.empty(E + 1, **i32) if expert_offsets is None else expert_offsets
+    sorted_pair = torch.empty(P, **i32) if sorted_pair is None else sorted_pair
+    pair_row = torch.empty(P, **i32) if pair_row is None else pair_row
+    _check(lib().moe_route_permute(
+        _ptr(logits, torch.float32, "logits"), T, E, k, _ptr(topk_idx, torch.int32),
+        _ptr(topk_w, torch.float32), _ptr(expert_offsets, torch.int32),
+        _ptr(sorted_pair, torch.int32), _ptr(pair_row, torch.int32), _stream(stream)),
+        "moe_route_permute")
+    return topk_idx, topk_w, expert_offsets, sorted_pair, pair_row
 
 
 def mxfp4_moe_ffn_workspace_bytes(T, k, H, I):

@@ -23,6 +23,7 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 0;
   bool greedy_attr = false;   // non-portable cluster size allowed for greedy_kernel
+  bool permute_attr = false;  // 33*1024 ints of dynamic shared memory for the permutation
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -86,6 +87,34 @@ const char *moe_status_string(int status) {
 
 int moe_version(void) { return 10000; }
 
+// Dynamic shared memory of the one-CTA permutation (33*E ints, E <= 1024),
+// set once per device for both kernels that run it.
+static int permute_attributes() {
+  DeviceInfo *dev = const_cast<DeviceInfo *>(device_info());
+  if (!dev) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!dev->permute_attr) {
+    const int bytes = 33 * 1024 * (int)sizeof(int);
+    if (cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(route_permute_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
+      return launch_status();
+    dev->permute_attr = true;
+  }
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ route --
 int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
                    float *topk_w, moe_stream_t stream) {
@@ -114,13 +143,38 @@ int moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *expert_of
   if (!expert_offsets) return MOE_ERR_INVALID_ARG;
   if (P > 0 && (!topk_idx || !sorted_pair || !pair_row)) return MOE_ERR_INVALID_ARG;
   const size_t smem = (size_t)33 * E * sizeof(int);
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         33 * 1024 * (int)sizeof(int));
-  });
+  const int st = permute_attributes();
+  if (st != MOE_OK) return st;
   return launched(launch_pdl(permute_kernel, 1, 1024, smem, (cudaStream_t)stream, topk_idx, (int)P,
                              E, expert_offsets, sorted_pair, pair_row));
+}
+
+// ---------------------------------------------------- route + permute --
+int moe_route_permute(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
+                      int32_t *expert_offsets, int32_t *sorted_pair, int32_t *pair_row,
+                      moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
+  if ((long long)T * k > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_idx || !topk_w || !sorted_pair || !pair_row))
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0 || T > ROUTE_PERMUTE_MAX_T) {
+    const int st = moe_route_topk(logits, T, E, k, topk_idx, topk_w, stream);
+    if (st != MOE_OK) return st;
+    return moe_permute(topk_idx, T, k, E, expert_offsets, sorted_pair, pair_row, stream);
+  }
+  const int st = permute_attributes();
+  if (st != MOE_OK) return st;
+  const size_t smem = (size_t)33 * E * sizeof(int);
+  auto kern = E <= 32    ? route_permute_kernel<1>
+              : E <= 64  ? route_permute_kernel<2>
+              : E <= 128 ? route_permute_kernel<4>
+              : E <= 256 ? route_permute_kernel<8>
+              : E <= 512 ? route_permute_kernel<16>
+                         : route_permute_kernel<32>;
+  return launched(launch_pdl(kern, 1, 1024, smem, (cudaStream_t)stream, logits, T, E, k, topk_idx,
+                             topk_w, expert_offsets, sorted_pair, pair_row));
 }
 
 // -------------------------------------------------------------------- FFN --

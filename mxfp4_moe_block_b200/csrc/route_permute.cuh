@@ -15,14 +15,9 @@ namespace moe {
 // owner lane marks it taken.  Weights: softmax of the selected logits in
 // double, summed in slot order, rounded once to float.
 template <int PER>
-__global__ void __launch_bounds__(128)
-route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
-                  int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
-  pdl_wait();
-  pdl_trigger();
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
+__device__ __forceinline__ void route_one_token(const float *__restrict__ logits, int t, int E,
+                                                int k, int lane, int32_t *topk_idx,
+                                                float *topk_w) {
   const float *row = logits + (size_t)t * E;
   float v[PER];
   unsigned taken = 0;
@@ -58,6 +53,18 @@ route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
   }
 }
 
+template <int PER>
+__global__ void __launch_bounds__(128)
+route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
+                  int32_t *__restrict__ topk_idx, float *__restrict__ topk_w) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  route_one_token<PER>(logits, t, E, k, lane, topk_idx, topk_w);
+}
+
 // Stable counting sort of P = T*k pairs by expert in one CTA of 1024 threads.
 // Warp w owns the contiguous pair range [w*seg, (w+1)*seg).
 //   pass A: per-warp, per-expert running counts; each pair's rank inside its
@@ -67,13 +74,12 @@ route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
 //           per-expert totals gives expert_offsets;
 //   pass C: pos = offset[e] + warp_base[w][e] + local rank.
 // Dynamic shared memory: 32*E counters + E offsets (ints).
-__global__ void __launch_bounds__(1024)
-permute_kernel(const int32_t *__restrict__ topk_idx, int P, int E,
-               int32_t *__restrict__ expert_offsets,
-               int32_t *__restrict__ sorted_pair, int32_t *__restrict__ pair_row) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ int smem[];
+// topk_idx is read with plain loads: the fused kernel below writes it in
+// the same launch.
+__device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, int E,
+                                              int32_t *__restrict__ expert_offsets,
+                                              int32_t *__restrict__ sorted_pair,
+                                              int32_t *__restrict__ pair_row, int *smem) {
   int *cnt = smem;             // [32][E]
   int *offs = smem + 32 * E;   // [E]
   __shared__ int warp_tot[32];
@@ -151,6 +157,36 @@ permute_kernel(const int32_t *__restrict__ topk_idx, int P, int E,
       }
     }
   }
+}
+
+__global__ void __launch_bounds__(1024)
+permute_kernel(const int32_t *__restrict__ topk_idx, int P, int E,
+               int32_t *__restrict__ expert_offsets,
+               int32_t *__restrict__ sorted_pair, int32_t *__restrict__ pair_row) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int smem[];
+  permute_block(topk_idx, P, E, expert_offsets, sorted_pair, pair_row, smem);
+}
+
+// Routing and permutation of a small batch in one CTA: warp w routes tokens
+// w, w + 32, ...; after the barrier the block's own global writes of
+// topk_idx are visible to it and the permutation runs as above.  One launch
+// instead of two on the verify step's critical path.
+constexpr int ROUTE_PERMUTE_MAX_T = 128;
+template <int PER>
+__global__ void __launch_bounds__(1024, 1)
+route_permute_kernel(const float *__restrict__ logits, int T, int E, int k,
+                     int32_t *topk_idx, float *__restrict__ topk_w,
+                     int32_t *__restrict__ expert_offsets, int32_t *__restrict__ sorted_pair,
+                     int32_t *__restrict__ pair_row) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ int smem[];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int t = w; t < T; t += 32) route_one_token<PER>(logits, t, E, k, lane, topk_idx, topk_w);
+  __syncthreads();
+  permute_block(topk_idx, T * k, E, expert_offsets, sorted_pair, pair_row, smem);
 }
 
 }  // namespace moe

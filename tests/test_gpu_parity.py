@@ -55,6 +55,44 @@ def test_route_permute_bit_exact(name):
         assert mm.moe_get_device_status() == (0, 0)
 
 
+@pytest.mark.parametrize("name", ALL)
+def test_fused_route_permute_matches_oracle(name):
+    """moe_route_permute (one kernel up to 128 tokens, two launches above)
+    gives the oracle's routing and grouping bit for bit."""
+    sh = synth.SHAPES[name]
+    L = Layer(sh, 0, DEV, with_weights=False)
+    idx, w, off, sp, pr = mm.moe_route_permute(L.logits, sh.k)
+    ridx, _, rw64 = omoe.route_topk(L.logits_np, sh.k)
+    roff, rsp, rpr = omoe.permute(ridx, sh.E)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert_route_weights(w.cpu().numpy(), rw64)
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.array_equal(sp.cpu().numpy(), rsp)
+    assert np.array_equal(pr.cpu().numpy(), rpr)
+    assert mm.moe_get_device_status() == (0, 0)
+
+
+def test_fused_route_permute_edges():
+    """Ties, signed zeros, one expert, k = E, E = 1024 and k = 32, every
+    routing width, T at and around the one-kernel limit, and an empty batch."""
+    rng = np.random.default_rng(11)
+    pool = np.array([-0.0, 0.0, 1.0, -2.5, 3.0], np.float32)
+    for T, E, k in [(1, 1, 1), (33, 5, 5), (128, 8, 3), (129, 8, 3), (17, 1024, 32),
+                    (40, 300, 7), (64, 64, 8), (100, 600, 4), (7, 32, 2)]:
+        l = pool[rng.integers(0, 5, (T, E))]
+        idx, w, off, sp, pr = mm.moe_route_permute(torch.from_numpy(l).to(DEV), k)
+        ridx, _, rw64 = omoe.route_topk(l, k)
+        roff, rsp, rpr = omoe.permute(ridx, E)
+        assert np.array_equal(idx.cpu().numpy(), ridx), (T, E, k)
+        assert_route_weights(w.cpu().numpy(), rw64)
+        assert np.array_equal(off.cpu().numpy(), roff), (T, E, k)
+        assert np.array_equal(sp.cpu().numpy(), rsp), (T, E, k)
+        assert np.array_equal(pr.cpu().numpy(), rpr), (T, E, k)
+    idx, w, off, sp, pr = mm.moe_route_permute(torch.zeros((0, 6), device=DEV), 2)
+    assert off.cpu().tolist() == [0] * 7
+    assert mm.moe_get_device_status() == (0, 0)
+
+
 def test_route_ties_signed_zero_and_max_sizes():
     rng = np.random.default_rng(5)
     for T, E, k in [(33, 1, 1), (64, 5, 5), (100, 8, 3), (17, 1024, 32), (40, 300, 7)]:

@@ -958,19 +958,25 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           for (int j = 0; j < kTokPerLd; ++j)
             if (tok0 + j < ntok) a.y[(size_t)(rtok0 + tok0 + j) * a.H + m] = tok_sum[j];
         } else {
-          // rows 0-63 gate (quarters 0,1), 64-127 up (quarters 2,3)
-          if (q >= 2) {
+          // Rows 0-63 gate (quarters 0,1), 64-127 up (quarters 2,3).  Quarter
+          // q and q+2 hold gate and up of the same 32 rows n; the gate warp
+          // finishes the chunk's even tokens, the up warp the odd ones, each
+          // handing the other its half through disjoint slots of xchg.
+          const int qq = q & 1;
+          const bool gate = q < 2;
+          const int slot0 = (32 * qq + lane) * 8;
 #pragma unroll
-            for (int j = 0; j < kTokPerLd; ++j) xchg[(32 * (q - 2) + lane) * 8 + j] = tok_sum[j];
-          }
+          for (int j = 0; j < kTokPerLd; ++j)
+            if ((j & 1) == (gate ? 1 : 0)) xchg[slot0 + j] = tok_sum[j];
           asm volatile("bar.sync 1, 128;" ::: "memory");
-          if (q < 2) {
-            const int n = mt * 64 + 32 * q + lane;
+          {
+            const int n = mt * 64 + 32 * qq + lane;
 #pragma unroll
             for (int j = 0; j < kTokPerLd; ++j) {
+              if ((j & 1) != (gate ? 0 : 1)) continue;
               const int tok = tok0 + j;
-              const float g = tok_sum[j];
-              const float u = xchg[(32 * q + lane) * 8 + j];
+              const float g = gate ? tok_sum[j] : xchg[slot0 + j];
+              const float u = gate ? xchg[slot0 + j] : tok_sum[j];
               const uint16_t hb = f32_to_bf16_bits(g / (1.f + expf(-g)) * u);
               const bool valid = tok < ntok;
               const size_t r = (size_t)(rtok0 + tok);

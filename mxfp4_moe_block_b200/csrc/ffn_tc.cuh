@@ -410,6 +410,81 @@ encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restric
   }
 }
 
+// The same encoding with one warp per row, for rows of K = 64 * PPL <= 2048
+// elements (PPL pairs per lane in registers, the row maximum by shuffles, no
+// block barrier): four rows per CTA (small CTAs stay resident beside a GEMM
+// CTA).  Same outputs as the kernel above.
+template <int NT, int PPL>
+__global__ void __launch_bounds__(128)
+encode_rows_f4_warp_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp,
+                           int k, int P, uint8_t *__restrict__ q, float *__restrict__ rs,
+                           int early_trigger, int *counters) {
+  if (early_trigger) pdl_trigger();
+  pdl_wait();
+  if (!early_trigger) pdl_trigger();
+  if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
+  constexpr int K = 64 * PPL;
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (r >= P) return;
+  const uint32_t *row =
+      reinterpret_cast<const uint32_t *>(src + (size_t)(sp ? __ldg(sp + r) / k : r) * K);
+  float v[2 * PPL];
+#pragma unroll
+  for (int j = 0; j < PPL; ++j) {
+    const uint32_t pr = __ldg(row + lane + 32 * j);
+    v[2 * j] = bf16_lo(pr);
+    v[2 * j + 1] = bf16_hi(pr);
+  }
+#pragma unroll 1
+  for (int t = 0; t < NT; ++t) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2 * PPL; ++j) m = fmaxf(m, fabsf(v[j]));
+    const float amax = warp_max(m);
+    const int sexp = amax > 0.f ? e2m1_block_exp(amax) : 0;
+    const float inv = pow2f(-sexp), sc = pow2f(sexp);
+    uint8_t *qrow = q + (size_t)(NT * r + t) * (K / 2);
+#pragma unroll
+    for (int j = 0; j < PPL; ++j) {
+      const uint32_t c0 = to_e2m1(v[2 * j] * inv), c1 = to_e2m1(v[2 * j + 1] * inv);
+      const float2 d = e2m1x2_to_f32x2(c0 | (c1 << 4));
+      v[2 * j] -= d.x * sc;
+      v[2 * j + 1] -= d.y * sc;
+      qrow[lane + 32 * j] = (uint8_t)(c0 | (c1 << 4));
+    }
+    if (lane == 0) rs[NT * r + t] = sc;
+  }
+}
+
+// Launch a row encoder: a CTA per row (shortest latency: a row's work
+// spread over 256 threads) for a few rows, a warp per row (no barriers, the
+// most rows per SM) once there are hundreds.
+constexpr size_t ENC_WARP_MIN_ROWS = 512;
+template <int NT>
+inline cudaError_t launch_encode_f4(const uint16_t *src, const int32_t *sp, int k, int K,
+                                   size_t P, uint8_t *q, float *rs, int early_trigger,
+                                   int *counters, cudaStream_t s) {
+  const unsigned g4 = (unsigned)((P + 3) / 4);
+  switch (P >= ENC_WARP_MIN_ROWS ? K : 0) {
+    case 256:
+      return launch_pdl(encode_rows_f4_warp_kernel<NT, 4>, g4, 128, 0, s, src, sp, k, (int)P, q,
+                        rs, early_trigger, counters);
+    case 512:
+      return launch_pdl(encode_rows_f4_warp_kernel<NT, 8>, g4, 128, 0, s, src, sp, k, (int)P, q,
+                        rs, early_trigger, counters);
+    case 1024:
+      return launch_pdl(encode_rows_f4_warp_kernel<NT, 16>, g4, 128, 0, s, src, sp, k, (int)P, q,
+                        rs, early_trigger, counters);
+    case 2048:
+      return launch_pdl(encode_rows_f4_warp_kernel<NT, 32>, g4, 128, 0, s, src, sp, k, (int)P, q,
+                        rs, early_trigger, counters);
+    default:
+      return launch_pdl(encode_rows_f4_kernel<NT>, (unsigned)P, ENC_THREADS, 0, s, src, sp, k, K,
+                        q, rs, early_trigger, counters);
+  }
+}
+
 // ------------------------------------------------------------- the kernel --
 
 struct TcMaps {
@@ -1100,8 +1175,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
                          C::kSmem);
   }
   if (KIND == KIND_F4) {
-    if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.x, f.sp, f.k, H, xq,
-                   reinterpret_cast<float *>(xs), 0, counters) != cudaSuccess)
+    if (launch_encode_f4<T>(f.x, f.sp, f.k, H, P, xq, reinterpret_cast<float *>(xs), 0, counters,
+                            s) != cudaSuccess)
       return MOE_ERR_CUDA;
   } else {
     const long blocks = (long)P * (H / 32);
@@ -1139,9 +1214,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
     return MOE_ERR_CUDA;
 
   if (KIND == KIND_F4)
-    if (launch_pdl(encode_rows_f4_kernel<T>, (unsigned)P, ENC_THREADS, 0, s, f.h,
-                   (const int32_t *)nullptr, 1, I, hq, reinterpret_cast<float *>(hs), 1,
-                   (int *)nullptr) != cudaSuccess)
+    if (launch_encode_f4<T>(f.h, nullptr, 1, I, P, hq, reinterpret_cast<float *>(hs), 1, nullptr,
+                            s) != cudaSuccess)
       return MOE_ERR_CUDA;
   // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;

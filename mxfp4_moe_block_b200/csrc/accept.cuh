@@ -24,7 +24,8 @@ namespace moe {
 namespace cg = cooperative_groups;
 
 constexpr int GREEDY_THREADS = 256;
-constexpr int GREEDY_UNROLL = 8;         // 16-byte loads in flight per thread
+constexpr int GREEDY_UNROLL = 10;        // 16-byte loads in flight per thread (a 152K-entry row
+                                         // slice of 1/16 in one round)
 constexpr int GREEDY_MAX_CLUSTER = 16;   // CTAs per row (non-portable cluster size)
 constexpr int GREEDY_TOKEN_BITS = 26;    // key = row << 26 | token; V <= 2^26
 constexpr unsigned GREEDY_NO_MISS = 0xffffffffu;

@@ -227,6 +227,13 @@ __device__ __forceinline__ void tc_st_x8(uint32_t taddr, const uint32_t (&r)[8])
 }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Named barrier of one epilogue warp group (ids 1 and 2, 128 threads each);
+// constant ids keep the kernel's barrier count small.
+__device__ __forceinline__ void group_sync(int grp) {
+  if (grp) asm volatile("bar.sync 2, 128;" ::: "memory");
+  else asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
@@ -307,6 +314,12 @@ struct TcKindCfg {
   static constexpr int kMmaK = kStageK / 4;                     // 4 MMAs per stage
   static constexpr uint32_t kABytes = 128u * kStageK / 2;       // packed weight bytes per stage
   static constexpr int kBRowBytesPerK2 = KIND == KIND_F4 ? 1 : 2;  // B row bytes = K * this / 2
+  // Epilogue warp groups (alternating 16-column chunks): two where tiles are
+  // wide and the SwiGLU work per tile is large; one for kind::mxf4, whose
+  // narrow tiles leave room for the encode kernels' CTAs beside the GEMM CTA.
+  static constexpr int kEpiGroups = KIND == KIND_F8 ? 2 : 1;
+  static constexpr int kThreads = (8 + 4 * kEpiGroups) * 32;
+  static constexpr int kRingReaders = 1 + 1 + 4 * kEpiGroups + 4;
   static constexpr bool kRowScaledB = KIND == KIND_F4;          // B scales per row, not block
 };
 
@@ -524,7 +537,8 @@ struct TcCfg {
   static constexpr int kSfb = Kd::kRowScaledB ? 0 : 512 * Kd::kKGroups * kRowChunks;
   static constexpr int kSfbConst = Kd::kRowScaledB ? 512 * kRowChunks : 0;  // all 1.0
   static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
-  static constexpr int kFixed = 1024 + 2048 + 1026 * 2 + 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
+  static constexpr int kFixed = 1024 + Kd::kEpiGroups * 64 * (16 / Kd::kTerms) * 4 + 1026 * 2 +
+                                 2 * 1025 * 4 + 128 + 1024 + kSfbConst;
   static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
   static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
   static constexpr int kSfCols =                                    // TMEM columns per stage
@@ -543,8 +557,11 @@ struct TcCfg {
   static constexpr int kOffSfa = kOffB + kStages * kB;
   static constexpr int kOffSfb = kOffSfa + kStages * kSfa;
   static constexpr int kOffBar = kOffSfb + kStages * kSfb;
-  static constexpr int kOffXchg = kOffBar + 1024;                // 64 rows x 4 tokens (float)
-  static constexpr int kOffTab = kOffXchg + 2048;                 // active list + prefix
+  // SwiGLU exchange: 64 rows x (tokens per 16-column chunk) floats per
+  // epilogue warp group
+  static constexpr int kXchgFloats = 64 * (16 / Kd::kTerms);
+  static constexpr int kOffXchg = kOffBar + 1024;
+  static constexpr int kOffTab = kOffXchg + Kd::kEpiGroups * kXchgFloats * 4;  // tile table
   // tile table: expert ids (16-bit), tile prefix and first sorted row (32-bit)
   static constexpr int kTabBytes = 1026 * 2 + 2 * 1025 * 4;
   static constexpr int kOffSfbConst = (kOffTab + kTabBytes + 127) & ~127;  // 16B-aligned for tcgen05.cp
@@ -555,10 +572,9 @@ struct TcCfg {
 };
 
 // warps: 0 TMA producer, 1 scale loader, 2 TMEM + MMA issuer, 3 constant B
-// scales, 4-7 epilogue, 8-11 A-scale writers (one per TMEM lane quarter)
-constexpr int TC_THREADS = 384;
+// scales, 4-7 epilogue, 8-11 scale writers (one per TMEM lane quarter),
+// 12-15 second epilogue group (kind::mxf8f6f4)
 constexpr int kRing = 4;                        // tile indices published ahead
-constexpr int kRingReaders = 1 + 1 + 4 + 4;
 
 // Reader side of the tile ring: tile i of this CTA's sequence (all lanes of
 // the calling warp wait; `arrive` is the one lane that releases the slot).
@@ -574,7 +590,7 @@ __device__ __forceinline__ int ring_read(uint64_t *ring_full, uint64_t *ring_emp
 }
 
 template <int KIND, int MODE, int BN>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TcKindCfg<KIND>::kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   using C = TcCfg<KIND, BN>;
   using Kd = TcKindCfg<KIND>;
@@ -643,11 +659,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&ring_full[r], 1);             // producer
-      mbar_init(&ring_empty[r], kRingReaders); // scale loader, MMA, 4 epilogue, 4 writers
+      mbar_init(&ring_empty[r], Kd::kRingReaders); // scale loader, MMA, epilogue, 4 writers
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);     // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], 4 * Kd::kEpiGroups);   // one arrival per epilogue warp
     }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -914,7 +930,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         tc_commit(&acc_full[buf]);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------- A-scale writers --
     // Warp 8+q stores lane quarter q of every stage's A scale columns with
     // tcgen05.st (the scale-factor layout repeats the same 32 lanes in all
@@ -956,9 +972,13 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------- epilogue --
-    // accumulator column T*j + t holds term t of token j of the tile
-    const int q = warp - 4;                     // TMEM lane quarter
+    // accumulator column T*j + t holds term t of token j of the tile.  Two
+    // groups of four warps (4-7 and 12-15, one per TMEM lane quarter each)
+    // take alternate 16-column chunks.
+    const int q = warp & 3;                     // TMEM lane quarter
+    const int grp = warp >= 12 ? 1 : 0;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    float *gx = xchg + grp * C::kXchgFloats;
     pdl_wait();                                 // row scales in, h / y out
     constexpr int kTokPerLd = 16 / T;           // tokens per 16-column load
     int it = 0;
@@ -972,18 +992,25 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       const int rtok0 = rowB / T;               // sorted row of the tile's first token
       // the first chunk's row scales do not depend on the accumulator: load
       // them while the MMAs still run
+      const int cfirst = 16 * grp;              // this group's first chunk
       float rs0[16];
       if (Kd::kRowScaledB) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int tok = min(i / T, ntok - 1);          // rows past ntok are discarded
+          const int tok = min((cfirst + i) / T, ntok - 1);   // rows past ntok are discarded
           rs0[i] = __ldg(a.b_rowscale + (size_t)(rtok0 + tok) * T + i % T);
         }
       }
       if (!mbar_wait_fast(&acc_full[buf], use & 1, abort)) break;
       tc_fence_after();
       const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
-      for (int c0 = 0; c0 < nB; c0 += 16) {
+      if (cfirst >= nB) {
+        // no chunk for this group: hand the buffer back at once
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+      for (int c0 = cfirst; c0 < nB; c0 += 16 * Kd::kEpiGroups) {
         float v[16];
         {
           uint32_t r[C::kChains][16];
@@ -999,7 +1026,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             v[i] = acc;
           }
         }
-        if (c0 + 16 >= nB) {
+        if (c0 + 16 * Kd::kEpiGroups >= nB) {
           // every accumulator column of the tile is in registers: hand the
           // buffer back to the MMA warp before the arithmetic and the stores
           tc_fence_before();
@@ -1012,7 +1039,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         for (int j = 0; j < kTokPerLd; ++j) {
           float sum = 0.f;
           if (Kd::kRowScaledB) {
-            if (c0 == 0) {
+            if (c0 == cfirst) {
 #pragma unroll
               for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], rs0[T * j + u], sum);
             } else {
@@ -1039,19 +1066,19 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           // handing the other its half through disjoint slots of xchg.
           const int qq = q & 1;
           const bool gate = q < 2;
-          const int slot0 = (32 * qq + lane) * 8;
+          const int slot0 = (32 * qq + lane) * kTokPerLd;
 #pragma unroll
           for (int j = 0; j < kTokPerLd; ++j)
-            if ((j & 1) == (gate ? 1 : 0)) xchg[slot0 + j] = tok_sum[j];
-          asm volatile("bar.sync 1, 128;" ::: "memory");
+            if ((j & 1) == (gate ? 1 : 0)) gx[slot0 + j] = tok_sum[j];
+          group_sync(grp);
           {
             const int n = mt * 64 + 32 * qq + lane;
 #pragma unroll
             for (int j = 0; j < kTokPerLd; ++j) {
               if ((j & 1) != (gate ? 0 : 1)) continue;
               const int tok = tok0 + j;
-              const float g = gate ? tok_sum[j] : xchg[slot0 + j];
-              const float u = gate ? xchg[slot0 + j] : tok_sum[j];
+              const float g = gate ? tok_sum[j] : gx[slot0 + j];
+              const float u = gate ? gx[slot0 + j] : tok_sum[j];
               const uint16_t hb = f32_to_bf16_bits(g / (1.f + expf(-g)) * u);
               const bool valid = tok < ntok;
               const size_t r = (size_t)(rtok0 + tok);
@@ -1061,7 +1088,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                                lane, valid);
             }
           }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
+          group_sync(grp);
         }
       }
     }
@@ -1210,7 +1237,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.b_rowscale = reinterpret_cast<const float *>(xs);
   a.K = H;
   a.rows_per_expert = 2 * I;
-  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, TC_THREADS, C::kSmem, s, maps, a) != cudaSuccess)
+  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps, a) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   if (KIND == KIND_F4)
@@ -1229,7 +1256,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.K = I;
   a.rows_per_expert = H;
   a.tile_counter = counters + 1;
-  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, TC_THREADS, C::kSmem, s, maps, a) != cudaSuccess)
+  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, Kd::kThreads, C::kSmem, s, maps, a) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

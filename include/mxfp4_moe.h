@@ -27,6 +27,16 @@
  *    by moe_get_device_status; the kernel then skips the offending element
  *    and never faults.  Inputs with NaN or infinity are unsupported: results
  *    are unspecified, but no fault occurs.
+ *  - Every kernel is launched with programmatic stream serialisation
+ *    (programmatic dependent launch): the next kernel on the stream may
+ *    become resident while the current one finishes, and waits for it
+ *    (griddepcontrol.wait) before it reads the current one's output or writes
+ *    anything.  A library kernel lets its successor launch only after its own
+ *    wait, so when a kernel starts early everything two launches back is
+ *    complete; kernels rely on that only for data the same call or the call
+ *    before produced (the FFN's second GEMM reads the expert offsets before
+ *    its wait).  Ordinary kernels of the caller are unaffected: without the
+ *    attribute a kernel waits for full completion as usual.
  */
 #ifndef MXFP4_MOE_H
 #define MXFP4_MOE_H

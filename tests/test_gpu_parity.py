@@ -185,8 +185,10 @@ def test_ffn_tensor(name, variant):
 
 def test_ffn_tensor_small_shapes_and_bn_classes():
     """tcgen05 path on small shapes: one expert with many rows (several B
-    tiles, a ragged last one) and every B-tile width class."""
-    for K, E, k in [(1, 4, 1), (37, 4, 1), (64, 2, 2), (200, 2, 1), (8, 64, 8)]:
+    tiles, a ragged last one), every B-tile width class, and 512+ pairs (the
+    warp-per-row activation encoder, for x and for h)."""
+    for K, E, k in [(1, 4, 1), (37, 4, 1), (64, 2, 2), (200, 2, 1), (8, 64, 8), (600, 4, 1),
+                    (260, 8, 2)]:
         sh = synth.Shape("tcs", H=512, I=256, E=E, k=k, S=1, K=K, V=64, seed=20 + K)
         L = Layer(sh, 0, DEV)
         idx, w, off, sp, pr = _route_permute(L, sh)

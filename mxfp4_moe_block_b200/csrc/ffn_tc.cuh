@@ -1,29 +1,31 @@
 // ffn_tc.cuh -- MXFP4 expert FFN on the 5th-generation tensor cores.
 //
 // The expert weights stay in their MXFP4 form all the way into the tensor
-// core: tcgen05.mma.kind::mxf8f6f4.block_scale takes A = E2M1 codes with one
-// E8M0 scale per 32 elements -- exactly the OCP MX block the pages name for
-// the experts ("MiMo-v2.5-Pro-UltraSpeed - infra 架构解读", section "FP4 Expert
+// core: the block-scaled tcgen05.mma takes A = E2M1 codes with one E8M0
+// scale per 32 elements -- exactly the OCP MX block the pages name for the
+// experts ("MiMo-v2.5-Pro-UltraSpeed - infra 架构解读", section "FP4 Expert
 // 量化"; "mimo-tilert-1000tps-trillion-parameter-inference", section
 // "第一层：FP4 选择性量化").  Nothing is dequantised on the CUDA cores.
 //
-// The activations (bf16) become the B operand as two E4M3 terms with their
-// own E8M0 block scales: x = s1*q1 + s2*q2 per 32-element block, q1 the
-// nearest E4M3 of x/s1, q2 that of the remainder.  A bf16 value has 8
-// significant bits and q1 captures the top 4, so the remainder is exact in
-// E4M3 whenever it stays in E4M3's normal range; what is lost is below
-// ~2^-18 of the block's largest element.  Each token occupies two adjacent
-// B rows (its two terms) and the epilogue adds the two accumulator columns.
+// The activations (bf16) become the B operand as a short sum of narrow terms
+// (see "activation block encodings" below): eight E2M1 terms with one scale
+// per row and term for kind::mxf4 (exact for bf16), or two E4M3 terms with
+// E8M0 block scales for kind::mxf8f6f4 (two B columns per token where tiles
+// are wide).
 //
-// One persistent CTA per SM walks a tile list (expert, 128-row block of the
-// weight matrix, block of B rows).  Warp roles, after the tile-pipelining and
+// One persistent CTA per SM takes tiles (expert, 128-row block of the weight
+// matrix, block of B rows): its first from blockIdx.x, the rest from an
+// atomic counter.  Warp roles, after the tile-pipelining and
 // warp-specialisation ideas the pages describe for TileRT (prior art):
-//   warp 0  TMA producer: weight tile (E2M1, 16U4_ALIGN16B so that each code
-//           lands in its own byte lane, 128B swizzle) + activation tile;
-//   warp 1  scale loader: cp.async of the scale bytes straight into the
-//           32-row x 16-byte layout tcgen05.cp wants;
-//   warp 2  TMEM allocation and the single MMA-issuing thread;
-//   warps 4-7 epilogue: TMEM -> registers -> SwiGLU (GEMM-1) or y (GEMM-2).
+//   warp 0     TMA producer: weight tile + activation tile per 16 KB stage,
+//              and the tile index ring every other role reads;
+//   warp 1     scale loader: cp.async of the scale bytes into shared memory
+//              in the 32-row x 16-byte layout of the scale-factor columns;
+//   warp 2     TMEM allocation and the single MMA-issuing thread;
+//   warp 3     constant B block scales (kind::mxf4);
+//   warps 4-7  epilogue: TMEM -> registers -> SwiGLU (GEMM-1) or y (GEMM-2);
+//   warps 8-11 scale writers: tcgen05.st of the stage's scale factors;
+//   warps 12-15 a second epilogue group (kind::mxf8f6f4).
 // Every wait is bounded; on time-out the kernel records MOE_DEV_TIMEOUT,
 // drains what it issued, frees its TMEM and returns.
 #pragma once
@@ -248,11 +250,15 @@ __device__ __forceinline__ float warp_max(float v) {
 //  * kind::mxf8f6f4: two E4M3 terms with an E8M0 scale per 32 elements
 //    (what is lost is below ~2^-18 of the block's largest element);
 //    warp-cooperative, lane l holds element l of one 32-element block.
-//  * kind::mxf4: four E2M1 terms with ONE scale per row and term, chosen
+//  * kind::mxf4: eight E2M1 terms with ONE scale per row and term, chosen
 //    from the row's largest remaining magnitude.  The MMA then sees a
 //    constant block scale of 1.0 for B (copied to tensor memory once per
 //    CTA), and the epilogue multiplies each term's column by its exact power
-//    of two.  Four terms leave ~1e-4 relative error in the dot products.
+//    of two.  Each term takes about two more significant bits of the
+//    largest remainder, so eight terms give bf16 rows back to ~1e-9
+//    relative (all but a few elements in 10^4 exactly), and each term
+//    column's fp32 sum over K -- products of E2M1 values and powers of two --
+//    rarely rounds: the FFN meets the oracle to ~1e-7.
 
 
 __device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(127 + s) << 23); }

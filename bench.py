@@ -65,11 +65,17 @@ def load_peaks():
 
 
 def kernel_source_tag():
+    """Hash of the CUDA sources' code (comments and blank lines left out), so a
+    committed traffic figure stays attached to the kernels it was taken on."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "mxfp4_moe_block_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        h.update(open(os.path.join(d, f), "rb").read())
+        text = open(os.path.join(d, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [ln.split("//", 1)[0].rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

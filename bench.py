@@ -115,6 +115,16 @@ def rank_shape(sh, rank):
     return synth.Shape(**{**sh.__dict__, "seed": sh.seed + 7919 * rank})
 
 
+def sum_over_ranks(value, world, device):
+    """All ranks' total (all-reduce SUM); identity on one rank."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def max_over_ranks(value, world, device):
     """Slowest rank's value (all-reduce MAX); identity on one rank."""
     if world <= 1:
@@ -476,6 +486,8 @@ def main():
     route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     tail_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     ms = max_over_ranks(ms, world, dev)
+    # draft tokens the step accepted (sum of accept_len over the sequences)
+    accepted = sum_over_ranks(int(wl.acc.sum().item()), world, dev)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h, e2e_mode = float("nan"), 0, 0, None
@@ -504,6 +516,7 @@ def main():
         "breakdown_ms": {"route+permute": route_ms, "ffn": ffn_ms, "combine+greedy": tail_ms,
                          "eager_step": eager_ms, "graph_step": ms if graph is not None else None},
         "ffn_tflops": wl.ffn_flops() / (ffn_ms * 1e-3) / 1e12,
+        "accepted_tokens_per_s": accepted / (ms * 1e-3),
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "timing": e2e_mode},
         "gpu_launches": launches_per_step * args.steps,

@@ -28,11 +28,12 @@ def _worker(rank, world, port, out):
     try:
         sh = synth.SHAPES["tiny"]
         mx = bench.max_over_ranks(1.5 + rank, world, "cpu")
+        tot = bench.sum_over_ranks(2 + rank, world, "cpu")
         shr = bench.rank_shape(sh, rank)
         x = synth.x_bf16_bits(shr)
         w = synth.weight_codes_np(sh, "w13", 0)
         cfg = bench.workload_config(sh, world)
-        out.put((rank, mx, int(x.astype("int64").sum()), int(w.astype("int64").sum()),
+        out.put((rank, mx, tot, int(x.astype("int64").sum()), int(w.astype("int64").sum()),
                  repr(sorted(cfg.items()))))
     finally:
         dist.destroy_process_group()
@@ -49,8 +50,9 @@ def test_two_ranks_max_time_and_distinct_batches():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, m0, x0, w0, c0), (r1, m1, x1, w1, c1) = res
+    (r0, m0, t0, x0, w0, c0), (r1, m1, t1, x1, w1, c1) = res
     assert m0 == m1 == 2.5                 # slowest rank's value on both
+    assert t0 == t1 == 5.0                 # all ranks' accepted tokens on both
     assert x0 != x1                        # different activations per rank
     assert w0 == w1                        # same weights
     assert c0 == c1 and "'global_batch_tokens', 16" in c0
@@ -60,3 +62,4 @@ def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.25, 1, "cpu") == 3.25
+    assert bench.sum_over_ranks(3.25, 1, "cpu") == 3.25

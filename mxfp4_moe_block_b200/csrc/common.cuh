@@ -86,10 +86,6 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p) {
   return r;
 }
 
-__device__ __forceinline__ uint4 ld_nc16(const void *p) {
-  return __ldg(reinterpret_cast<const uint4 *>(p));
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);

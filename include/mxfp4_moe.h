@@ -157,12 +157,15 @@ int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
 enum {
   MOE_FFN_AUTO = 0,      /* tensor cores if H >= 512, else FMA                   */
   MOE_FFN_FMA = 1,       /* dequantise to registers, float FMA                   */
-  MOE_FFN_TENSOR = 2,    /* tcgen05 block-scaled MMA: TENSOR_F4 if H, I are
-                            multiples of 256, else TENSOR_F8                      */
+  MOE_FFN_TENSOR = 2,    /* tcgen05 block-scaled MMA: TENSOR_F4 while its B
+                            tiles stay narrow (8*T*k <= 128 * min(T*k, E)) and
+                            H, I are multiples of 256 up to 8192, else
+                            TENSOR_F8                                             */
   MOE_FFN_TENSOR_F8 = 3, /* kind::mxf8f6f4: padded E2M1 weights x two E4M3
-                            activation terms                                      */
-  MOE_FFN_TENSOR_F4 = 4  /* kind::mxf4: packed E2M1 weights x four E2M1
-                            activation terms (H, I multiples of 256)              */
+                            activation terms with E8M0 block scales               */
+  MOE_FFN_TENSOR_F4 = 4  /* kind::mxf4: packed E2M1 weights x eight E2M1
+                            activation terms with one scale per row and term
+                            (H, I multiples of 256, at most 8192)                 */
 };
 
 /* Same contract as mxfp4_moe_ffn with an explicit kernel variant. */

@@ -1,0 +1,45 @@
+"""The benchmark's reference arm (the oracle, timed on the host) and its
+configuration text: host-only, no GPU."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_line_has_the_contract_keys():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny", "--steps", "2", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert line["steps"] == 2 and line["warmup"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_oracle_step_slices_the_expert_to_fit_a_budget():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mxfp4_moe_block_b200 import synth
+    step = bench.OracleStep(synth.SHAPES["tiny"])
+    full = step.i_s
+    step.fit(steps=10**6, budget_s=1e-3)         # an impossible budget: slice down
+    assert step.i_s < full and step.i_s % 32 == 0 and step.i_s >= 64 or full <= 64
+    assert step.run() > 0
+    assert f"{step.i_s} of its {full}" in step.sample_text()
+
+
+def test_l2_statement_follows_the_weight_bytes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from mxfp4_moe_block_b200 import synth
+    assert bench.l2_statement(synth.SHAPES["batch1"]).startswith("inputs larger than L2")
+    assert bench.l2_statement(synth.SHAPES["tiny"]).startswith("inputs smaller than L2")

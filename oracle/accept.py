@@ -24,6 +24,12 @@ this; the exact-arithmetic reading used here (identical on every device):
   R_0 + ... + R_v > m;
 * if S == 0 the same draw is taken from P_v = floor(p_v * 2**40);
 * all K accepted -> next token -1 (no bonus row).
+
+With a bonus row (the K+1 convention of speculative decoding: the target also
+scores the position after the block), all K accepted emits the target's own
+token for that position instead of -1: its argmax (greedy), or a draw from p
+at row K by the same integer rule on P_v (rejection).  `greedy_bonus` and
+`rejection_bonus` state that variant.
 """
 from __future__ import annotations
 
@@ -103,4 +109,57 @@ def rejection(p: np.ndarray, q: np.ndarray, draft: np.ndarray,
         acc[s] = a
         if a < K:
             nxt[s] = residual_sample(p[s, a], q[s, a], u_resample[s])
+    return acc, nxt
+
+
+def greedy_bonus(logits: np.ndarray, draft: np.ndarray):
+    """Greedy acceptance with a bonus row.  logits [S, K+1, V], draft [S, K].
+
+    Rows 0..K-1 check drafts 0..K-1 as in `greedy`; row K is the target's
+    prediction after the whole block.  Returns accept_len [S] in [0, K] and
+    next_token [S] = argmax of row accept_len (the bonus row when all K drafts
+    were accepted), never -1.
+    """
+    S, K1, _ = logits.shape
+    K = K1 - 1
+    if draft.shape != (S, K):
+        raise ValueError("draft must be [S, K] for logits [S, K+1, V]")
+    acc = np.zeros(S, dtype=np.int32)
+    nxt = np.zeros(S, dtype=np.int32)
+    for s in range(S):
+        a = K
+        for i in range(K):
+            if argmax_lowest(logits[s, i]) != int(draft[s, i]):
+                a = i
+                break
+        acc[s] = a
+        nxt[s] = argmax_lowest(logits[s, a])
+    return acc, nxt
+
+
+def bonus_sample(p_row: np.ndarray, u_resample: float) -> int:
+    """Token drawn from the target row p by the integer inverse-CDF rule."""
+    Pw = [int(v) for v in np.floor(p_row.astype(np.float64) * 2.0 ** 40)]
+    U = int(float(u_resample) * 2 ** 24)
+    if not 0 <= U < 2 ** 24:
+        raise ValueError("u_resample must lie in [0, 1)")
+    if sum(Pw) == 0:
+        raise ValueError("target row has no mass")
+    return _draw(Pw, U)
+
+
+def rejection_bonus(p: np.ndarray, q: np.ndarray, draft: np.ndarray,
+                    u_accept: np.ndarray, u_resample: np.ndarray):
+    """Rejection sampling with a bonus row.  p [S, K+1, V] (row K: the target
+    after the block), q [S, K, V], draft [S, K], u_accept [S, K], u_resample
+    [S].  As `rejection` on rows 0..K-1; when all K drafts are accepted the
+    next token is drawn from p[s, K] (`bonus_sample`) instead of -1."""
+    S, K1, _ = p.shape
+    K = K1 - 1
+    if q.shape[:2] != (S, K) or draft.shape != (S, K):
+        raise ValueError("q [S, K, V] and draft [S, K] for p [S, K+1, V]")
+    acc, nxt = rejection(p[:, :K], q, draft, u_accept, u_resample)
+    for s in range(S):
+        if acc[s] == K:
+            nxt[s] = bonus_sample(p[s, K], u_resample[s])
     return acc, nxt

@@ -143,3 +143,100 @@ def test_rejection_negative_control_fails_chi2(monkeypatch):
         return real(p_row, np.zeros_like(q_row), u)
     monkeypatch.setattr(accept, "residual_sample", wrong)
     assert _chi2_trials() > CHI2_CRIT_15DOF_P001
+
+
+# ------------------------------------------------------------ bonus row (K+1) --
+
+def test_greedy_bonus_brute_force_all_drafts():
+    """Every draft block over a 3-token vocabulary: the accepted prefix is the
+    longest run of argmax matches and the emitted token is the argmax of the
+    first unmatched row -- the bonus row K when all K match."""
+    rng = np.random.default_rng(31)
+    K, V = 3, 3
+    logits = rng.normal(size=(1, K + 1, V)).astype(np.float32)
+    am = logits[0].argmax(-1)
+    for code in range(V ** K):
+        d = np.array([(code // V ** i) % V for i in range(K)], np.int32)[None]
+        acc, nxt = accept.greedy_bonus(logits, d)
+        a = 0
+        while a < K and d[0, a] == am[a]:
+            a += 1
+        assert acc[0] == a and nxt[0] == am[a]
+
+
+def test_greedy_bonus_reduces_to_greedy_before_the_last_row():
+    rng = np.random.default_rng(32)
+    S, K, V = 64, 8, 50
+    logits = rng.normal(size=(S, K + 1, V)).astype(np.float32)
+    am = logits[:, :K].argmax(-1)
+    d = np.where(rng.random((S, K)) < 0.1, (am + 1) % V, am).astype(np.int32)
+    acc_b, nxt_b = accept.greedy_bonus(logits, d)
+    acc, nxt = accept.greedy(logits[:, :K], d)
+    assert np.array_equal(acc_b, acc)
+    part = acc < K
+    assert np.array_equal(nxt_b[part], nxt[part])
+    assert np.array_equal(nxt_b[~part], logits[~part, K].argmax(-1))
+    assert (~part).any() and part.any()
+
+
+def test_rejection_bonus_reduces_to_rejection_and_draws_from_p():
+    rng = np.random.default_rng(33)
+    S, K, V = 200, 4, 12
+    p = rng.random((S, K + 1, V)).astype(np.float32)
+    p /= p.sum(-1, keepdims=True)
+    q = p[:, :K].copy()                               # q == p: every draft accepted
+    d = rng.integers(0, V, (S, K)).astype(np.int32)
+    ua = rng.random((S, K)).astype(np.float32)
+    ur = (rng.integers(0, 2 ** 24, S) / 2 ** 24).astype(np.float32)
+    acc, nxt = accept.rejection_bonus(p, q, d, ua, ur)
+    assert (acc == K).all()
+    for s in range(S):
+        assert nxt[s] == accept.bonus_sample(p[s, K], ur[s])
+    q2 = rng.random((S, K, V)).astype(np.float32)
+    q2 /= q2.sum(-1, keepdims=True)
+    acc2, nxt2 = accept.rejection_bonus(p, q2, d, ua, ur)
+    acc1, nxt1 = accept.rejection(p[:, :K], q2, d, ua, ur)
+    assert np.array_equal(acc2, acc1)
+    part = acc1 < K
+    assert np.array_equal(nxt2[part], nxt1[part])
+
+
+def test_bonus_sample_boundaries():
+    p = np.zeros(5, np.float32)
+    p[1], p[3] = 0.25, 0.75
+    assert accept.bonus_sample(p, 0.0) == 1
+    assert accept.bonus_sample(p, 0.25 - 2 ** -24) == 1
+    assert accept.bonus_sample(p, 0.25) == 3
+    assert accept.bonus_sample(p, 1 - 2 ** -24) == 3
+
+
+def _bonus_chi2(draw_row, n=1_000_000, V=16, seed=78):
+    """Chi-square of 10^6 bonus draws from `draw_row(p)` against p."""
+    z = synth.normal_np(synth.stream_key(seed, "p_logits"), 0, V)
+    p = np.exp(z - z.max())
+    p = (p / p.sum()).astype(np.float32)
+    ur = synth.u24_np(synth.stream_key(seed, "u_resample"), 0, n)
+    row = draw_row(p)
+    Pw = np.floor(row.astype(np.float64) * 2.0 ** 40).astype(np.int64)
+    cum = np.cumsum(Pw)
+    U = (ur.astype(np.float64) * 2 ** 24).astype(np.int64)
+    m = (cum[-1].astype(object) * U.astype(object)) // 2 ** 24
+    draws = np.searchsorted(cum, np.array(m, dtype=np.int64), side="right")
+    # the vectorised draw is the oracle's rule: spot-check it against bonus_sample
+    for i in range(0, n, n // 50):
+        assert draws[i] == accept.bonus_sample(row, ur[i])
+    counts = np.bincount(draws, minlength=V)
+    expect = p.astype(np.float64) / p.astype(np.float64).sum() * n
+    return float(((counts - expect) ** 2 / expect).sum())
+
+
+def test_bonus_draw_follows_p_chi2():
+    """The bonus token of fully accepted blocks is distributed as the target's
+    row K: chi-square over 10^6 seeded draws, 15 dof, p >= 0.001."""
+    assert _bonus_chi2(lambda p: p) <= CHI2_CRIT_15DOF_P001
+
+
+def test_bonus_chi2_negative_control():
+    """A planted mistake -- the draw taken from the neighbouring token's
+    probability (an off-by-one row index) -- fails the same test."""
+    assert _bonus_chi2(lambda p: np.roll(p, 1)) > CHI2_CRIT_15DOF_P001

@@ -101,6 +101,36 @@ def encode_e2m1(x: np.ndarray, scale_byte: int) -> np.ndarray:
     return (best + 8 * neg).astype(np.uint8)
 
 
+def quantize_mxfp4(w: np.ndarray):
+    """Real matrix [R, K] (K a multiple of 32) -> MXFP4 (codes [R, K/2] uint8,
+    scales [R, K/32] uint8), by the OCP MX v1.0 conversion: per 32-element
+    block the shared scale is X = 2**(floor(log2(amax)) - 2) (2 = the largest
+    E2M1 exponent), clamped to the E8M0 range, and each element becomes the
+    nearest E2M1 code of v / X, ties to even, saturating at +-6.  An all-zero
+    block takes the smallest scale (byte 0).  This is the format's own
+    encoder, for a weight quantiser; the verify path never quantises."""
+    w = np.asarray(w, dtype=np.float64)
+    R, K = w.shape
+    if K % 32:
+        raise ValueError("K must be a multiple of 32")
+    if not np.isfinite(w).all():
+        raise ValueError("non-finite input")
+    codes = np.zeros((R, K), dtype=np.uint8)
+    scales = np.zeros((R, K // 32), dtype=np.uint8)
+    for r in range(R):
+        for b in range(K // 32):
+            blk = w[r, 32 * b:32 * b + 32]
+            amax = float(np.abs(blk).max())
+            if amax == 0.0:
+                byte = 0
+            else:
+                _, ex = math.frexp(amax)              # amax = m * 2**ex, m in [0.5, 1)
+                byte = min(254, max(0, (ex - 1) - 2 + 127))
+            scales[r, b] = byte
+            codes[r, 32 * b:32 * b + 32] = encode_e2m1(blk, byte)
+    return pack_codes(codes), scales
+
+
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round float64 values to the nearest bfloat16 (ties to even), as float64.
 

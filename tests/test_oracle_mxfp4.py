@@ -113,3 +113,57 @@ def test_bf16_bits_round_trip():
 def test_dequantize_rejects_bad_scale_shape():
     with pytest.raises(ValueError):
         mxfp4.dequantize(np.zeros((2, 16), np.uint8), np.zeros((2, 2), np.uint8))
+
+
+# ------------------------------------------------- OCP MX conversion (encoder) --
+
+def test_quantize_scale_is_floor_log2_minus_two():
+    w = np.zeros((1, 64))
+    w[0, 5] = 6.0           # floor(log2 6) = 2 -> X = 2**0
+    w[0, 40] = -0.7         # floor(log2 0.7) = -1 -> X = 2**-3
+    c, s = mxfp4.quantize_mxfp4(w)
+    assert list(s[0]) == [127, 124]
+    assert mxfp4.dequantize(c, s)[0, 5] == 6.0
+    assert mxfp4.dequantize(c, s)[0, 40] == -0.75   # 0.7 / 2**-3 = 5.6 -> 6
+
+
+def test_quantize_value_round_trip_of_mxfp4_matrices():
+    """Any MXFP4 matrix's values survive quantisation exactly (the scale may
+    change when a block's largest code is below 4, the values may not)."""
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, (16, 64 // 2), dtype=np.uint8)
+    scales = rng.integers(110, 140, (16, 64 // 32), dtype=np.uint8)
+    v = mxfp4.dequantize(codes, scales)
+    c2, s2 = mxfp4.quantize_mxfp4(v)
+    assert np.array_equal(mxfp4.dequantize(c2, s2), v)
+
+
+def test_quantize_error_bound_and_nearest_code():
+    """Per block 4X <= amax < 8X; an element within +-6X becomes the nearest
+    representable value (brute force over the 16 codes), one beyond
+    saturates to +-6X; so |q - w| <= 2X."""
+    rng = np.random.default_rng(6)
+    w = rng.normal(size=(8, 96)) * np.exp(rng.normal(size=(8, 1)) * 3)
+    c, s = mxfp4.quantize_mxfp4(w)
+    q = mxfp4.dequantize(c, s)
+    for r in range(8):
+        for b in range(3):
+            X = 2.0 ** (int(s[r, b]) - 127)
+            blk, qb = w[r, 32 * b:32 * b + 32], q[r, 32 * b:32 * b + 32]
+            assert 4 * X <= np.abs(blk).max() < 8 * X
+            assert np.abs(qb - blk).max() <= 2 * X
+            inside = np.abs(blk) <= 6 * X
+            cands = mxfp4.E2M1_TABLE[None, :] * X
+            nearest = np.abs(blk[:, None] - cands).min(axis=1)
+            assert np.array_equal(np.abs(qb - blk)[inside], nearest[inside])
+            assert np.array_equal(qb[~inside], np.sign(blk[~inside]) * 6 * X)
+
+
+def test_quantize_zero_block_and_bad_input():
+    c, s = mxfp4.quantize_mxfp4(np.zeros((2, 32)))
+    assert (s == 0).all() and (mxfp4.dequantize(c, s) == 0).all()
+    import pytest
+    with pytest.raises(ValueError):
+        mxfp4.quantize_mxfp4(np.zeros((1, 33)))
+    with pytest.raises(ValueError):
+        mxfp4.quantize_mxfp4(np.full((1, 32), np.inf))

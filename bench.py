@@ -1,14 +1,19 @@
 """Benchmark of the MXFP4 MoE block-verify step on B200.
 
-One step = the whole hot path over one drafted batch: moe_route_topk ->
-moe_permute -> mxfp4_moe_ffn -> moe_combine -> block_accept_greedy (the
-batch-1 verify workload: 1 sequence x 8-token block, one MoE layer of
+One step = the whole hot path over one drafted batch: moe_route_permute ->
+mxfp4_moe_ffn -> moe_combine (per MoE layer; stacked layers add a
+moe_rms_norm before and the residual in the combine) -> block acceptance
+(block_accept_greedy and/or block_accept_rejection).  The headline line is
+the batch-1 verify workload (1 sequence x 8-token block, one MoE layer of
 hidden 7168, expert intermediate 2048, 256 experts, top-8; greedy acceptance
 over a 152064-token vocabulary).  Metric: verified tokens/s (= S*K / step
-time), with the HBM roofline of the expert FFN beside it.
+time), with the expert FFN's roofline beside it.  On one GPU the same line
+carries `per_config`: the other seeded workloads (tiny, serving batch, DFlash
+block-16 with rejection acceptance, the 8-layer stack) each timed the same
+way with its own roofline, plus the MXFP4 weight quantiser.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload batch1|serving|tiny]
+                    [--workload NAME] [--no-per-config] [--no-cpu-baseline]
 
 Multi-GPU: every rank verifies its own independent batch (the path has no
 exchange step); value = all ranks' tokens / the slowest rank's time.
@@ -18,6 +23,7 @@ on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import json
 import os
 import shutil
@@ -37,36 +43,40 @@ from mxfp4_moe_block_b200 import synth  # noqa: E402
 
 METRIC = "verified tokens/s (MXFP4 MoE block-verify step)"
 UNIT = "tokens/s"
+PER_CONFIG = ("tiny", "serving", "dflash16", "multilayer")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    # the step times one MoE layer with greedy acceptance: the configurations
-    # of that form; the others (rejection acceptance, stacked layers) are
-    # parity-test cases
-    ap.add_argument("--workload", default="batch1",
-                    choices=[n for n, s in synth.SHAPES.items()
-                             if s.layers == 1 and s.accept == ("greedy",)])
+    ap.add_argument("--workload", default="batch1", choices=list(synth.SHAPES))
     ap.add_argument("--variant", type=int, default=0, help="FFN kernel: 0 auto, 1 FMA, 2 tensor")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--per-config", default=",".join(PER_CONFIG),
+                    help="comma-separated workloads for the per_config object")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the expert count (smaller cases for profiler captures)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def load_peaks():
+    """Roofline denominators: the machine's measured copy bandwidth and dense bf16
+    GEMM rate (MEASURED_PEAKS.json), else the earlier measurement on this machine."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
     except Exception:
-        return 6650.0, "fallback"
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
 
 
 def kernel_source_tag():
@@ -104,7 +114,8 @@ def load_traffic(workload, variant_name):
 def workload_config(sh, world):
     """The `config` object of the JSON line (identical for both arms)."""
     acc = " + ".join(sh.accept)
-    layers = f"{sh.layers} stacked MoE layers" if sh.layers > 1 else "one MoE layer"
+    layers = (f"{sh.layers} stacked MoE layers (RMSNorm, residual)" if sh.layers > 1
+              else "one MoE layer")
     return {
         "workload": f"{sh.name}: {layers} H={sh.H} I={sh.I} E={sh.E} top-{sh.k} SwiGLU, "
                     f"S={sh.S} x K={sh.K} block, {acc} acceptance over V={sh.V}",
@@ -122,7 +133,7 @@ def l2_statement(sh):
     does not flush L2 between steps; it relies on that)."""
     # expected distinct experts when P pairs pick among E uniformly
     experts = sh.E * (1.0 - (1.0 - 1.0 / sh.E) ** sh.P)
-    gb = experts * sh.expert_bytes() / 1e9
+    gb = experts * sh.expert_bytes() * sh.layers / 1e9
     if experts * sh.expert_bytes() > L2_BYTES:
         return f"inputs larger than L2: ~{gb:.2f} GB of MXFP4 expert weights read per step"
     return (f"inputs smaller than L2 (~{gb * 1e3:.1f} MB of expert weights, no flush): "
@@ -156,14 +167,17 @@ def max_over_ranks(value, world, device):
 
 
 class ClockSampler:
+    """nvidia-smi clock samples, taken only while a timed region runs
+    (start/stop may be called several times; the samples accumulate)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = None
+        self.sm, self.mx, self.reasons = [], 0.0, set()
 
     def start(self):
         if shutil.which("nvidia-smi") is None:
@@ -179,86 +193,134 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         time.sleep(0.25)
         self.proc.terminate()
         self.proc.wait(timeout=10)
+        self.proc = None
         self.f.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
+                self.sm.append(float(parts[1]))
+                self.mx = max(self.mx, float(parts[2]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(self.NAMES, parts[5:9]):
                 if v.lower().startswith("active"):
-                    reasons.add(n)
+                    self.reasons.add(n)
         os.unlink(self.path)
-        if not sm:
+
+    def summary(self):
+        if not self.sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.mx,
+                "reasons": sorted(self.reasons), "samples": len(self.sm)}
 
 
 # ------------------------------------------------------------------ workload --
 
+def _i32(n, device):
+    return torch.empty(n, dtype=torch.int32, device=device)
+
+
 class Workload:
-    """Seeded inputs of one verify step, resident in HBM."""
+    """Seeded inputs and buffers of one verify step, resident in HBM.
+
+    Layer l of a stack: xn = rms_norm(residual) (layer 0 reads x), route and
+    permute its router logits, the expert FFN, and a combine that adds the
+    residual; a single layer combines without residual.  Then the block
+    acceptance the workload names."""
 
     def __init__(self, sh, device, rank):
         import mxfp4_moe_block_b200 as mm
         self.mm = mm
         self.sh = sh
         self.dev = device
-        self.sh_r = rank_shape(sh, rank)
-        s = self.sh_r
+        s = self.sh_r = rank_shape(sh, rank)
+        T, k, E, H, I, L = s.T, s.k, s.E, s.H, s.I, s.layers
         self.x_bits = synth.x_bf16_bits(s)
-        self.logits_np = synth.router_logits(s)
-        self.block_np = synth.block_logits(s)
-        self.draft_np = synth.greedy_drafts(s, self.block_np)
         self.x = torch.from_numpy(self.x_bits.view(np.int16)).to(device).view(torch.bfloat16)
-        self.logits = torch.from_numpy(self.logits_np).to(device)
-        self.block = torch.from_numpy(self.block_np).to(device)
-        self.draft = torch.from_numpy(self.draft_np).to(device)
-        self.w = synth.weights_torch(sh, 0, device)      # model weights: same on every rank
-        T, k, E, H, I = s.T, s.k, s.E, s.H, s.I
-        i32 = dict(dtype=torch.int32, device=device)
-        self.idx = torch.empty((T, k), **i32)
+        self.logits_np = [synth.router_logits(s, l) for l in range(L)]
+        self.logits = [torch.from_numpy(a).to(device) for a in self.logits_np]
+        self.w = [synth.weights_torch(sh, l, device) for l in range(L)]   # same on every rank
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.tw = torch.empty((T, k), dtype=torch.float32, device=device)
-        self.off = torch.empty(E + 1, **i32)
-        self.sp = torch.empty(T * k, **i32)
-        self.pr = torch.empty(T * k, **i32)
+        self.off = [_i32(E + 1, device) for _ in range(L)]
+        self.sp = _i32(T * k, device)
+        self.pr = _i32(T * k, device)
         self.y = torch.empty((T * k, H), dtype=torch.float32, device=device)
         self.ws = mm.alloc_workspace(T, k, H, I, device)
-        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-        self.acc = torch.empty(s.S, **i32)
-        self.nxt = torch.empty(s.S, **i32)
+        self.xn = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+        # outputs the caller reads back, packed in one buffer: the combined
+        # hidden states, then accept lengths and next tokens per acceptance
+        self.greedy = "greedy" in s.accept
+        self.rejection = "rejection" in s.accept
+        nacc = int(self.greedy) + int(self.rejection)
+        out_bytes = T * H * 2
+        self.result = torch.empty(out_bytes + nacc * 2 * s.S * 4, dtype=torch.uint8, device=device)
+        self.out = self.result[:out_bytes].view(torch.bfloat16).view(T, H)
+        acc_views = self.result[out_bytes:].view(torch.int32).view(nacc, 2, s.S)
+        j = 0
+        if self.greedy:
+            self.block_np = synth.block_logits(s)
+            self.draft_np = synth.greedy_drafts(s, self.block_np)
+            self.block = torch.from_numpy(self.block_np).to(device)
+            self.draft = torch.from_numpy(self.draft_np).to(device)
+            self.acc_g, self.nxt_g = acc_views[j, 0], acc_views[j, 1]
+            j += 1
+        if self.rejection:
+            ri = synth.rejection_inputs(s)
+            self.rej = [torch.from_numpy(np.ascontiguousarray(a)).to(device)
+                        for a in (ri.p, ri.q, ri.draft, ri.u_accept, ri.u_resample)]
+            self.acc_r, self.nxt_r = acc_views[j, 0], acc_views[j, 1]
 
     def step(self, variant, ev=None):
+        """One verify step; `ev` (optional) = CUDA events: ev['ffn'][l] a
+        (start, end) pair around layer l's FFN, ev['start'] / ev['end']."""
         mm, s = self.mm, self.sh_r
+        L = s.layers
         if ev is not None:
-            ev[0].record()
-        mm.moe_route_permute(self.logits, s.k, s.E, self.idx, self.tw, self.off, self.sp, self.pr)
+            ev["start"].record()
+        for l in range(L):
+            if L > 1:
+                mm.moe_rms_norm(self.x if l == 0 else self.out, out=self.xn)
+                xin = self.xn
+            else:
+                xin = self.x
+            mm.moe_route_permute(self.logits[l], s.k, s.E, self.idx, self.tw, self.off[l],
+                                 self.sp, self.pr)
+            if ev is not None:
+                ev["ffn"][l][0].record()
+            mm.mxfp4_moe_ffn(xin, s.k, *self.w[l], self.off[l], self.sp, y=self.y,
+                             workspace=self.ws, variant=variant)
+            if ev is not None:
+                ev["ffn"][l][1].record()
+            if L > 1:
+                mm.moe_combine(self.y, self.pr, self.tw, residual=self.x if l == 0 else self.out,
+                               out=self.out)
+            else:
+                mm.moe_combine(self.y, self.pr, self.tw, out=self.out)
+        if self.greedy:
+            mm.block_accept_greedy(self.block, self.draft, self.acc_g, self.nxt_g)
+        if self.rejection:
+            mm.block_accept_rejection(*self.rej, self.acc_r, self.nxt_r)
         if ev is not None:
-            ev[1].record()
-        mm.mxfp4_moe_ffn(self.x, s.k, *self.w, self.off, self.sp, y=self.y, workspace=self.ws,
-                         variant=variant)
-        if ev is not None:
-            ev[2].record()
-        mm.moe_combine(self.y, self.pr, self.tw, out=self.out)
-        mm.block_accept_greedy(self.block, self.draft, self.acc, self.nxt)
-        if ev is not None:
-            ev[3].record()
+            ev["end"].record()
 
-    def activated_bytes(self):
-        off = self.off.cpu().numpy()
-        n_act = int((np.diff(off) > 0).sum())
-        return n_act * self.sh.expert_bytes(), n_act
+    def active_experts(self):
+        return [int((np.diff(o.cpu().numpy()) > 0).sum()) for o in self.off]
+
+    def accepted(self):
+        """Draft tokens accepted in the last step, per acceptance kind."""
+        out = {}
+        if self.greedy:
+            out["greedy"] = int(self.acc_g.sum().item())
+        if self.rejection:
+            out["rejection"] = int(self.acc_r.sum().item())
+        return out
 
     def ffn_flops(self):
         return 2.0 * self.sh_r.P * 3 * self.sh.H * self.sh.I
@@ -277,45 +339,254 @@ def count_launches(wl, variant):
     return len(names), sorted(set(names))
 
 
+def capture_graph(wl, variant):
+    """One step captured as a CUDA graph (launch gaps removed)."""
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        wl.step(variant)
+    torch.cuda.current_stream().wait_stream(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        wl.step(variant)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    return graph
+
+
+def time_steps(wl, variant, steps, warmup, use_graph, clocks=None, barrier=lambda: None):
+    """Device time of `steps` steps (CUDA events on the launching stream,
+    synchronised on both sides), then an eager pass with events around each
+    FFN call for the per-call breakdown."""
+    for _ in range(max(3, warmup)):
+        wl.step(variant)
+    torch.cuda.synchronize()
+    graph = capture_graph(wl, variant) if use_graph else None
+    if clocks:
+        clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            wl.step(variant)
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = a.elapsed_time(b) / steps
+    L = wl.sh.layers
+    evs = [{"start": torch.cuda.Event(enable_timing=True), "end": torch.cuda.Event(enable_timing=True),
+            "ffn": [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(L)]} for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        wl.step(variant, evs[i])
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.stop()
+    eager_ms = statistics.mean(e["start"].elapsed_time(e["end"]) for e in evs)
+    ffn_ms = [statistics.mean(e["ffn"][l][0].elapsed_time(e["ffn"][l][1]) for e in evs)
+              for l in range(L)]
+    del graph
+    return {"ms": ms, "eager_ms": eager_ms, "ffn_ms": ffn_ms,
+            "timing": "CUDA graph replay" if use_graph else "eager"}
+
+
+def roofline(wl, ffn_ms, peaks, variant_name):
+    """The expert FFN against its two rooflines (per layer, averaged): the
+    active experts' MXFP4 bytes over the measured copy bandwidth, and the
+    FFN's FLOPs over the measured dense bf16 GEMM rate.  `bound` is the
+    roofline with the longer time; frac = that time / the measured time."""
+    sh = wl.sh
+    act = wl.active_experts()
+    bytes_l = [n * sh.expert_bytes() for n in act]
+    flops = wl.ffn_flops()
+    ms = statistics.mean(ffn_ms)
+    byts = statistics.mean(bytes_l)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9) * 1e3
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+    hbm = {"achieved_gbs": byts / (ms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+           "frac": t_hbm / ms, "algorithmic_bytes": byts, "active_experts": act}
+    tc = {"achieved_tflops": flops / (ms * 1e-3) / 1e12, "peak_tflops": peaks["bf16_tflops"],
+          "frac": t_tc / ms, "flops": flops,
+          "peak_note": "dense bf16 (activations are bf16; the MMAs run block-scaled "
+                       "fp8/fp4 kinds on exact narrow terms of them)"}
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    traffic = load_traffic(sh.name, variant_name)
+    return {"bound": bound,
+            "achieved": hbm["achieved_gbs"] if bound == "hbm" else tc["achieved_tflops"],
+            "peak": hbm["peak_gbs"] if bound == "hbm" else tc["peak_tflops"],
+            "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": max(t_hbm, t_tc) / ms, "traffic": traffic,
+            "kernel": "mxfp4_moe_ffn (encode, GEMM-1+SwiGLU, encode, GEMM-2 launches)",
+            "ffn_ms": ms, "hbm": hbm, "tensor": tc,
+            "peak_source": f"{peaks['source']} hbm_gbs / bf16_tflops"}
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+class OracleSample:
+    """The oracle on a bounded sample of one verify step: the first `n_tok`
+    tokens of the batch through every layer -- their routing over all E
+    experts, the permutation, the SwiGLU FFN of each of their (token, expert)
+    pairs, the combine and, for stacked layers, the RMSNorm and residual --
+    then the acceptance of the sequences those tokens belong to.  Tokens are
+    independent inside an MoE layer (router logits are given), so this is
+    exactly the step's work for those tokens.  Inputs, expert weights
+    included, are drawn before timing.  `workers` > 1 runs the (token,
+    expert) FFNs of a layer on a thread pool (numpy releases the GIL) with one
+    BLAS thread each; 1 is the plain single-thread oracle."""
+
+    def __init__(self, sh, n_tok, workers=1):
+        from oracle import moe as omoe
+        self.sh = sh
+        self.n_tok = n_tok = max(1, min(n_tok, sh.T))
+        self.workers = workers
+        self.toks = np.arange(n_tok)
+        self.seqs = (0, (n_tok - 1) // sh.K + 1)
+        x = synth.bf16_bits_to_f32(synth.x_bf16_bits(sh)).astype(np.float64)
+        self.x64 = x[self.toks]
+        self.logits = [synth.router_logits(sh, l)[self.toks] for l in range(sh.layers)]
+        self.W = []
+        for l in range(sh.layers):
+            idx, _, _ = omoe.route_topk(self.logits[l], sh.k)
+            self.W.append({int(e): (synth.weight_codes_np(sh, "w13", int(e), l),
+                                    synth.weight_scales_np(sh, "w13", int(e), l),
+                                    synth.weight_codes_np(sh, "w2", int(e), l),
+                                    synth.weight_scales_np(sh, "w2", int(e), l))
+                           for e in np.unique(idx)})
+        if "greedy" in sh.accept:
+            self.block = synth.block_logits(sh, seqs=self.seqs)
+            self.draft = synth.greedy_drafts(sh, self.block, seqs=self.seqs)
+        if "rejection" in sh.accept:
+            self.ri = synth.rejection_inputs(sh, seqs=self.seqs)
+
+    def run(self):
+        from threadpoolctl import threadpool_limits
+
+        from oracle import accept as oacc
+        from oracle import moe as omoe
+        sh = self.sh
+        pool = (concurrent.futures.ThreadPoolExecutor(max_workers=self.workers)
+                if self.workers > 1 else None)
+        try:
+            with threadpool_limits(limits=1):
+                t0 = time.perf_counter()
+                r = self.x64
+                for l in range(sh.layers):
+                    xn = omoe.rms_norm(r) if sh.layers > 1 else r
+                    idx, w, _ = omoe.route_topk(self.logits[l], sh.k)
+                    off, sp, pr = omoe.permute(idx, sh.E)
+                    y = np.zeros((len(sp), sh.H))
+                    jobs = [(e, int(off[e]), int(off[e + 1])) for e in range(sh.E)
+                            if off[e + 1] > off[e]]
+
+                    def one(job, xn=xn, sp=sp, l=l):
+                        e, r0, r1 = job
+                        _, ye = omoe.expert_ffn(xn[sp[r0:r1] // sh.k], *self.W[l][e], sh.I)
+                        return r0, r1, ye
+                    for r0, r1, ye in (pool.map(one, jobs) if pool else map(one, jobs)):
+                        y[r0:r1] = ye
+                    r, _ = omoe.combine(y, pr, w, r if sh.layers > 1 else None)
+                if "greedy" in sh.accept:
+                    oacc.greedy(self.block, self.draft)
+                if "rejection" in sh.accept:
+                    ri = self.ri
+                    oacc.rejection(ri.p, ri.q, ri.draft, ri.u_accept, ri.u_resample)
+                return time.perf_counter() - t0
+        finally:
+            if pool:
+                pool.shutdown()
+
+    def text(self):
+        seq = self.seqs[1] - self.seqs[0]
+        return (f"{self.n_tok} of the step's {self.sh.T} tokens through all {self.sh.layers} "
+                f"layer(s) (routing, permutation, every expert FFN of those tokens, combine) "
+                f"and the acceptance of their {seq} sequence(s); inputs drawn before timing")
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def sample_tokens(sh, cores):
+    """Tokens in an oracle sample: the whole batch where its experts are small
+    (the tiny shape), else as many tokens as give every core one (token,
+    expert) FFN -- at least one."""
+    if sh.H * sh.I <= 1 << 20:
+        return sh.T
+    return max(1, min(sh.T, cores // sh.k))
+
+
+def cpu_baseline(sh):
+    """Oracle tokens/s on the host: single thread, and all cores."""
+    cores = host_cores()
+    one = OracleSample(sh, sample_tokens(sh, 1), workers=1)
+    t1 = one.run()
+    many = OracleSample(sh, sample_tokens(sh, cores), workers=cores)
+    tn = many.run()
+    return {"value": many.n_tok / tn, "unit": UNIT, "cores": min(cores, many.n_tok * sh.k),
+            "kind": "oracle", "sample": many.text(), "seconds": tn,
+            "single_core": {"value": one.n_tok / t1, "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": one.text(), "seconds": t1},
+            "host_cores": cores}
+
+
+# ---------------------------------------------------------------------- e2e --
+
 def e2e_time(wl, variant, steps, warmup):
     """The same step through the public API with host buffers, as a serving
-    loop runs it: every step's inputs are copied in from pinned host memory
-    and its results (combined hidden states, accept lengths, next tokens)
-    copied out, inside the timed region.  Each step (its kernels and the
-    copies out) is one CUDA graph; the copy in of step i+1 runs on a second
-    stream into the other of two input buffer sets while step i computes."""
-    hx = torch.from_numpy(wl.x_bits.view(np.int16)).pin_memory()
-    hl = torch.from_numpy(wl.logits_np).pin_memory()
-    hb = torch.from_numpy(wl.block_np).pin_memory()
-    hd = torch.from_numpy(wl.draft_np).pin_memory()
-    ho = torch.empty(wl.out.shape, dtype=torch.bfloat16).pin_memory()
-    ha = torch.empty(wl.acc.shape, dtype=torch.int32).pin_memory()
-    hn = torch.empty(wl.nxt.shape, dtype=torch.int32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hl, hb, hd))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, ha, hn))
-    # two input sets on the device: set 0 is the workload's own tensors
-    sets = [(wl.x, wl.logits, wl.block, wl.draft),
-            (torch.empty_like(wl.x), torch.empty_like(wl.logits), torch.empty_like(wl.block),
-             torch.empty_like(wl.draft))]
+    loop runs it: every step's inputs (x, router logits, block logits, drafts;
+    one pinned staging buffer) are copied in with one copy and its results
+    (combined hidden states, accept lengths, next tokens; one packed buffer)
+    copied out with one copy, inside the timed region.  Each step (its kernels
+    and the copy out) is one CUDA graph; the copy in of step i+1 runs on a
+    second stream into the other of two input buffer sets while step i
+    computes.  Also measures the host-to-device copy rate alone."""
+    arrays = [wl.x_bits.view(np.uint8), wl.logits_np[0].view(np.uint8),
+              wl.block_np.view(np.uint8), wl.draft_np.view(np.uint8)]
+    offs, o = [], 0
+    for a in arrays:
+        offs.append(o)
+        o += (a.nbytes + 255) // 256 * 256
+    host_in = torch.empty(o, dtype=torch.uint8).pin_memory()
+    for a, off in zip(arrays, offs):
+        host_in[off:off + a.nbytes] = torch.from_numpy(np.ascontiguousarray(a).reshape(-1))
+    h2d = sum(a.nbytes for a in arrays)
+    host_out = torch.empty(wl.result.numel(), dtype=torch.uint8).pin_memory()
+    d2h = wl.result.numel()
+    s = wl.sh_r
 
-    def copy_in(i):
-        x, lg, blk, dr = sets[i]
-        x.view(torch.int16).copy_(hx, non_blocking=True)
-        lg.copy_(hl, non_blocking=True)
-        blk.copy_(hb, non_blocking=True)
-        dr.copy_(hd, non_blocking=True)
+    def views(buf):
+        x = buf[offs[0]:offs[0] + arrays[0].nbytes].view(torch.bfloat16).view(s.T, s.H)
+        lg = buf[offs[1]:offs[1] + arrays[1].nbytes].view(torch.float32).view(s.T, s.E)
+        blk = buf[offs[2]:offs[2] + arrays[2].nbytes].view(torch.float32).view(s.S, s.K, s.V)
+        dr = buf[offs[3]:offs[3] + arrays[3].nbytes].view(torch.int32).view(s.S, s.K)
+        return x, lg, blk, dr
+    bufs = [torch.empty(o, dtype=torch.uint8, device=wl.dev) for _ in range(2)]
+    sets = [views(b) for b in bufs]
+    saved = (wl.x, wl.logits[0], wl.block, wl.draft)
+
+    def use(i):
+        wl.x, wl.logits[0], wl.block, wl.draft = sets[i]
 
     def step_out(i):
-        wl.x, wl.logits, wl.block, wl.draft = sets[i]
+        use(i)
         wl.step(variant)
-        ho.copy_(wl.out, non_blocking=True)
-        ha.copy_(wl.acc, non_blocking=True)
-        hn.copy_(wl.nxt, non_blocking=True)
+        host_out.copy_(wl.result, non_blocking=True)
 
     compute = torch.cuda.current_stream()
     copy = torch.cuda.Stream()
     for i in (0, 1):
-        copy_in(i)
+        bufs[i].copy_(host_in, non_blocking=True)
         step_out(i)
     torch.cuda.synchronize()
     graphs = []
@@ -330,14 +601,13 @@ def e2e_time(wl, variant, steps, warmup):
         with torch.cuda.graph(g):
             step_out(i)
         graphs.append(g)
-    wl.x, wl.logits, wl.block, wl.draft = sets[0]
     ev_in = [torch.cuda.Event(), torch.cuda.Event()]
     ev_done = [torch.cuda.Event(), torch.cuda.Event()]
 
     def run(n):
         copy.wait_stream(compute)
         with torch.cuda.stream(copy):
-            copy_in(0)
+            bufs[0].copy_(host_in, non_blocking=True)
             ev_in[0].record(copy)
         for i in range(n):
             cur, nxt = i % 2, 1 - i % 2
@@ -345,7 +615,7 @@ def e2e_time(wl, variant, steps, warmup):
                 if i >= 1:
                     copy.wait_event(ev_done[nxt])     # step i-1 has read set nxt
                 with torch.cuda.stream(copy):
-                    copy_in(nxt)
+                    bufs[nxt].copy_(host_in, non_blocking=True)
                     ev_in[nxt].record(copy)
             compute.wait_event(ev_in[cur])
             graphs[cur].replay()
@@ -358,119 +628,108 @@ def e2e_time(wl, variant, steps, warmup):
     run(steps)
     b.record(compute)
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / steps, h2d, d2h, "CUDA graph per step, copy-in of the next step overlapped"
+    ms = a.elapsed_time(b) / steps
+    # the host link alone: the step's input copy, and a large pinned copy
+    link = {}
+    for name, n in (("step_input", o), ("256MiB", 256 << 20)):
+        hsrc = host_in if n == o else torch.empty(n, dtype=torch.uint8).pin_memory()
+        dst = torch.empty(n, dtype=torch.uint8, device=wl.dev)
+        with torch.cuda.stream(copy):
+            for _ in range(3):
+                dst.copy_(hsrc, non_blocking=True)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(copy)
+            for _ in range(10):
+                dst.copy_(hsrc, non_blocking=True)
+            e1.record(copy)
+        torch.cuda.synchronize()
+        link[f"h2d_gbs_{name}"] = 10 * n / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    wl.x, wl.logits[0], wl.block, wl.draft = saved
+    del graphs
+    return ms, h2d, d2h, link
 
 
-# --------------------------------------------------------------- CPU oracle --
+# ---------------------------------------------------------------- quantiser --
 
-def oracle_step_seconds(sh, n_expert_sample=4, seed_shift=0):
-    """Time the CPU oracle on one step of the workload, with the expert FFN
-    on a sample of the active experts, scaled to all of them."""
-    from threadpoolctl import threadpool_limits
-
-    from oracle import accept as oacc
-    from oracle import moe as omoe
-    s = synth.Shape(**{**sh.__dict__, "seed": sh.seed + seed_shift})
-    x64 = synth.bf16_bits_to_f32(synth.x_bf16_bits(s)).astype(np.float64)
-    logits = synth.router_logits(s)
-    block = synth.block_logits(s)
-    draft = synth.greedy_drafts(s, block)
-    with threadpool_limits(limits=1):
-        t0 = time.perf_counter()
-        idx, w, _ = omoe.route_topk(logits, s.k)
-        off, sp, pr = omoe.permute(idx, s.E)
-        t_route = time.perf_counter() - t0
-        act = [e for e in range(s.E) if off[e + 1] > off[e]]
-        sample = act[:: max(1, len(act) // n_expert_sample)][:n_expert_sample]
-        y = np.zeros((s.P, s.H))
-        t_ffn = 0.0
-        for e in sample:
-            r0, r1 = off[e], off[e + 1]
-            wts = (synth.weight_codes_np(s, "w13", e), synth.weight_scales_np(s, "w13", e),
-                   synth.weight_codes_np(s, "w2", e), synth.weight_scales_np(s, "w2", e))
-            t0 = time.perf_counter()            # weights are inputs: drawn before timing
-            _, y[r0:r1] = omoe.expert_ffn(x64[sp[r0:r1] // s.k], *wts, s.I)
-            t_ffn += time.perf_counter() - t0
-        t_ffn *= len(act) / len(sample)
-        t0 = time.perf_counter()
-        omoe.combine(y, pr, w)
-        oacc.greedy(block, draft)
-        t_rest = time.perf_counter() - t0
-    total = t_route + t_ffn + t_rest
-    return total, {"experts_active": len(act), "experts_sampled": len(sample)}
+def measure_quantize(device, peaks, reps=10):
+    """mxfp4_quantize on 16 experts' worth of W13 rows ([16*4096, 7168] bf16,
+    0.94 GB, larger than L2) against the copy-bandwidth roofline."""
+    import mxfp4_moe_block_b200 as mm
+    R, K = 16 * 4096, 7168
+    g = torch.Generator(device=device)
+    g.manual_seed(1234)
+    w = (torch.randn((R, K), generator=g, device=device, dtype=torch.float32) * 0.02).to(torch.bfloat16)
+    codes = torch.empty((R, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((R, K // 32), dtype=torch.uint8, device=device)
+    for _ in range(3):
+        mm.mxfp4_quantize(w, codes, scales)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        mm.mxfp4_quantize(w, codes, scales)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    byts = R * K * (2 + 0.5 + 1 / 32)
+    gbs = byts / (ms * 1e-3) / 1e9
+    del w, codes, scales
+    return {"kernel": "mxfp4_quantize_kernel", "shape": [R, K], "ms": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": byts,
+                         "traffic": None}}
 
 
-class OracleStep:
-    """The reference arm's step: the oracle (one thread) on the step's inputs,
-    drawn once.  Routing, permutation, combine and greedy acceptance run in
-    full; the expert FFN runs for one active expert on the first `i_s` of
-    its I intermediate units (the SwiGLU of an I-slice is the same oracle
-    code on fewer gate/up/down rows), and its time is scaled by
-    (active experts) x I / i_s.  `i_s` is chosen so that the whole run of
-    steps fits the time budget."""
+# --------------------------------------------------------------- per config --
 
-    def __init__(self, sh):
-        from oracle import moe as omoe
-        self.sh = sh
-        self.x64 = synth.bf16_bits_to_f32(synth.x_bf16_bits(sh)).astype(np.float64)
-        self.logits = synth.router_logits(sh)
-        self.block = synth.block_logits(sh)
-        self.draft = synth.greedy_drafts(sh, self.block)
-        idx, _, _ = omoe.route_topk(self.logits, sh.k)
-        off, _, _ = omoe.permute(idx, sh.E)
-        self.active = [e for e in range(sh.E) if off[e + 1] > off[e]]
-        e = self.active[len(self.active) // 2]
-        self.expert = e
-        self.w13c = synth.weight_codes_np(sh, "w13", e)
-        self.w13s = synth.weight_scales_np(sh, "w13", e)
-        self.w2c = synth.weight_codes_np(sh, "w2", e)
-        self.w2s = synth.weight_scales_np(sh, "w2", e)
-        self.i_s = sh.I
+def measure_config(name, variant, steps, warmup, device, peaks, clocks, with_cpu):
+    sh = synth.SHAPES[name]
+    wl = Workload(sh, device, 0)
+    t = time_steps(wl, variant, steps, warmup, True, clocks)
+    n_launch, _ = count_launches(wl, variant)
+    acc = wl.accepted()
+    vname = {0: "auto", 1: "fma", 2: "tensor"}.get(variant, str(variant))
+    entry = {
+        "config": workload_config(sh, 1),
+        "ms_per_step": t["ms"], "timing": t["timing"],
+        "verified_tokens_per_s": sh.T / (t["ms"] * 1e-3),
+        "accepted_tokens_per_s": {k: v / (t["ms"] * 1e-3) for k, v in acc.items()},
+        "ffn_ms_per_layer": statistics.mean(t["ffn_ms"]),
+        "eager_ms_per_step": t["eager_ms"],
+        "roofline": roofline(wl, t["ffn_ms"], peaks, vname),
+        "launches_per_step": n_launch,
+    }
+    del wl
+    torch.cuda.empty_cache()
+    if with_cpu:
+        entry["cpu_baseline"] = cpu_baseline(sh)
+    return entry
 
-    def _slice(self, i_s):
-        I = self.sh.I
-        rows = np.r_[0:i_s, I:I + i_s]
-        return (self.w13c[rows], self.w13s[rows], self.w2c[:, :i_s // 2],
-                self.w2s[:, :i_s // 32])
 
-    def run(self):
-        from threadpoolctl import threadpool_limits
+# ---------------------------------------------------------------- reference --
 
-        from oracle import accept as oacc
-        from oracle import moe as omoe
-        sh, i_s = self.sh, self.i_s
-        wts = self._slice(i_s)
-        with threadpool_limits(limits=1):
-            t0 = time.perf_counter()
-            idx, w, _ = omoe.route_topk(self.logits, sh.k)
-            off, sp, pr = omoe.permute(idx, sh.E)
-            t_route = time.perf_counter() - t0
-            e = self.expert
-            r0, r1 = off[e], off[e + 1]
-            y = np.zeros((sh.P, sh.H))
-            t0 = time.perf_counter()
-            _, y[r0:r1] = omoe.expert_ffn(self.x64[sp[r0:r1] // sh.k], *wts, i_s)
-            t_ffn = (time.perf_counter() - t0) * len(self.active) * sh.I / i_s
-            t0 = time.perf_counter()
-            omoe.combine(y, pr, w)
-            oacc.greedy(self.block, self.draft)
-            t_rest = time.perf_counter() - t0
-        return t_route + t_ffn + t_rest
-
-    def fit(self, steps, budget_s):
-        """Shrink the I-slice until steps x (one step's wall time) fits."""
-        while True:
-            t0 = time.perf_counter()
-            self.run()
-            wall = time.perf_counter() - t0
-            if wall * steps <= budget_s or self.i_s <= 64:
-                return
-            self.i_s = max(64, (int(self.i_s * budget_s / (wall * steps)) // 32) * 32)
-
-    def sample_text(self):
-        return (f"route+permute+combine+greedy in full; expert FFN on 1 of "
-                f"{len(self.active)} active experts and {self.i_s} of its {self.sh.I} "
-                f"intermediate units, time scaled to all")
+def reference_arm(args, sh):
+    """The oracle as the reference arm, on the host cores: every step is a
+    real, timed bounded sample of the workload (OracleSample with all cores)."""
+    cores = host_cores()
+    samp = OracleSample(sh, sample_tokens(sh, cores), workers=cores)
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = samp.run()
+        if i >= args.warmup:
+            times.append(t)
+    ms = 1e3 * statistics.mean(times)
+    value = samp.n_tok / (ms / 1e3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": workload_config(sh, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(cores, samp.n_tok * sh.k),
+                         "kind": "oracle", "sample": samp.text()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
 
 
 # --------------------------------------------------------------------- main --
@@ -485,33 +744,14 @@ def main():
         sh = synth.Shape(**{**sh.__dict__, "E": args.experts, "name": f"{sh.name}-E{args.experts}"})
 
     if args.impl == "reference":
-        if rank != 0:
-            return
-        ostep = OracleStep(sh)
-        ostep.fit(args.warmup + args.steps, budget_s=150.0)   # the whole run: a few minutes
-        times = []
-        for i in range(args.warmup + args.steps):
-            t = ostep.run()
-            if i >= args.warmup:
-                times.append(t)
-        ms = 1e3 * statistics.mean(times)
-        value = sh.T / (ms / 1e3)
-        line = {
-            "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded counter-based generator)",
-            "config": workload_config(sh, 1),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": ostep.sample_text()},
-            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        }
-        print(json.dumps(line))
+        if rank == 0:
+            print(json.dumps(reference_arm(args, sh)))
         return
 
     if world > 1:
-        import torch.distributed as dist
         import datetime
+
+        import torch.distributed as dist
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
@@ -520,108 +760,67 @@ def main():
     dev = torch.device("cuda", local)
     import mxfp4_moe_block_b200 as mm
     mm.lib()
-    wl = Workload(sh, dev, rank)
+    peaks = load_peaks()
     variant = args.variant
-
-    for _ in range(max(3, args.warmup)):
-        wl.step(variant)
-    torch.cuda.synchronize()
-    act_bytes, n_act = wl.activated_bytes()
+    vname = {0: "auto", 1: "fma", 2: "tensor"}.get(variant, str(variant))
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    # CUDA graph of one step (launch gaps removed); eager launches otherwise
-    graph = None
-    if not args.no_graph:
-        stream = torch.cuda.Stream()
-        stream.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(stream):
-            wl.step(variant)
-        torch.cuda.current_stream().wait_stream(stream)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            wl.step(variant)
-        for _ in range(3):
-            graph.replay()
-        torch.cuda.synchronize()
-
     clocks = ClockSampler(local)
-    clocks.start()
-    barrier()
-    torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record()
-    for i in range(args.steps):
-        if graph is not None:
-            graph.replay()
-        else:
-            wl.step(variant)
-    t_end.record()
-    torch.cuda.synchronize()
-    barrier()
-    ms = t_start.elapsed_time(t_end) / args.steps
-    # per-call breakdown on eager launches, events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(args.steps):
-        wl.step(variant, evs[i])
-    e1.record()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    eager_ms = e0.elapsed_time(e1) / args.steps
-    ffn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    tail_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-    ms = max_over_ranks(ms, world, dev)
-    # draft tokens the step accepted (sum of accept_len over the sequences)
-    accepted = sum_over_ranks(int(wl.acc.sum().item()), world, dev)
+    wl = Workload(sh, dev, rank)
+    t = time_steps(wl, variant, args.steps, args.warmup, not args.no_graph, clocks, barrier)
+    ms = max_over_ranks(t["ms"], world, dev)
+    acc = wl.accepted()
+    accepted = sum_over_ranks(sum(acc.values()), world, dev)
 
-    if args.no_e2e:
-        e2e_ms, h2d, d2h, e2e_mode = float("nan"), 0, 0, None
+    # the host-buffer path is staged for the single-layer greedy workloads
+    e2e_ok = wl.sh.layers == 1 and wl.greedy and not wl.rejection
+    if args.no_e2e or not e2e_ok:
+        e2e_ms, h2d, d2h, link = float("nan"), 0, 0, {}
     else:
-        e2e_ms, h2d, d2h, e2e_mode = e2e_time(wl, variant, args.steps, 3)
+        e2e_ms, h2d, d2h, link = e2e_time(wl, variant, args.steps, 3)
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
-    peak, peak_kind = load_peaks()
-    achieved = act_bytes / (ffn_ms * 1e-3) / 1e9
-    vname = {0: "auto", 1: "fma", 2: "tensor"}[variant]
-    traffic = load_traffic(sh.name, vname)
     tokens = sh.T * world
     launches_per_step, kernel_names = count_launches(wl, variant)
     line = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4 weights, bf16 activations, f32 accumulate",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "mxfp4 weights, bf16 activations, f32 accumulate",
         "data": "synthetic (seeded counter-based generator; random MXFP4 weights)",
         "config": workload_config(sh, world),
-        "ffn_variant": vname, "timing": "CUDA graph replay" if graph is not None else "eager",
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "mxfp4_moe_ffn (GEMM-1+SwiGLU and GEMM-2 launches)",
-                     "algorithmic_bytes": act_bytes, "active_experts": n_act,
-                     "peak_source": f"{peak_kind} hbm_gbs"},
-        "breakdown_ms": {"route+permute": route_ms, "ffn": ffn_ms, "combine+greedy": tail_ms,
-                         "eager_step": eager_ms, "graph_step": ms if graph is not None else None},
-        "ffn_tflops": wl.ffn_flops() / (ffn_ms * 1e-3) / 1e12,
+        "ffn_variant": vname, "timing": t["timing"],
+        "roofline": roofline(wl, t["ffn_ms"], peaks, vname),
+        "breakdown_ms": {"ffn": statistics.mean(t["ffn_ms"]) * sh.layers,
+                         "rest": t["eager_ms"] - sum(t["ffn_ms"]),
+                         "eager_step": t["eager_ms"], "graph_step": t["ms"]},
+        "ffn_tflops": wl.ffn_flops() / (statistics.mean(t["ffn_ms"]) * 1e-3) / 1e12,
         "accepted_tokens_per_s": accepted / (ms * 1e-3),
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "timing": e2e_mode},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3) if e2e_ms == e2e_ms else None,
+                "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "timing": "CUDA graph per step, one copy in (overlapped with the previous step) "
+                          "and one copy out per step", **link},
         "gpu_launches": launches_per_step * args.steps,
         "launches_per_step": launches_per_step,
         "kernels": [n.split("(")[0].split("<")[0].replace("void ", "") for n in kernel_names],
-        "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, info = oracle_step_seconds(sh)
-        line["cpu_baseline"] = {
-            "value": sh.T / t, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"one step; expert FFN on {info['experts_sampled']} of "
-                      f"{info['experts_active']} active experts, time scaled to all"}
+    del wl
+    torch.cuda.empty_cache()
+    if world == 1:
+        if not args.no_per_config:
+            pc = {}
+            for name in [n for n in args.per_config.split(",") if n and n != sh.name]:
+                pc[name] = measure_config(name, variant, min(args.steps, 20), args.warmup, dev,
+                                          peaks, clocks, not args.no_cpu_baseline)
+            pc["quantize"] = measure_quantize(dev, peaks)
+            line["per_config"] = pc
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(sh)
+    line["clocks"] = clocks.summary()
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -93,6 +93,11 @@ int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
 
 /*
  * moe_permute -- stable grouping of the T*k (token, slot) pairs by expert.
+ *   The pages route each token to a few experts ([P4] "万亿参数推理为什么特别难")
+ *   and run the experts on the drafted block ([P3] "数据流概览"), but say
+ *   nothing about how the pairs are grouped or ordered.  Reading taken here:
+ *   a stable grouping, so that the order is unique and checkable --
+ *   experts ascending, pairs ascending by id inside an expert.
  *   Pair id p = t*k + j.  expert_offsets[e] .. expert_offsets[e+1] is the
  *   range of sorted rows of expert e; sorted_pair lists pair ids expert by
  *   expert, ascending inside an expert; pair_row is its inverse
@@ -214,6 +219,10 @@ int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
 
 /*
  * moe_combine -- weighted sum of each token's k expert outputs.
+ *   The pages do not state how expert outputs are merged ([P4]
+ *   "万亿参数推理为什么特别难" only says each token uses a few experts).
+ *   Reading taken here, the usual MoE combine with the routing weights of
+ *   moe_route_topk, in a fixed order so that results are reproducible:
  *   out[t] = bf16( sum_{j<k} topk_w[t,j] * y[pair_row[t*k+j]] + residual[t] )
  *   in float, slots summed in order j = 0..k-1, residual added last.
  *   y [T*k, H] float, pair_row [T*k], topk_w [T, k] float,
@@ -276,6 +285,60 @@ int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
                            int32_t *next_token, moe_stream_t stream);
 
 /*
+ * block_accept_greedy_bonus -- block_accept_greedy with a bonus row.
+ *   The target scores K + 1 positions per sequence: rows 0..K-1 check the K
+ *   drafts as in block_accept_greedy, row K is its prediction after the
+ *   whole block.  When every draft is accepted the target's own token for
+ *   that next position is emitted instead of -1, so each verify step yields
+ *   accept_len + 1 tokens (the target takes over after the last confirmed
+ *   token, [P2] "二、投机解码"; the drafter proposes a fixed-size block,
+ *   [P1] "接受率预测与动态回退机制").
+ *   next_token = argmax(logits[s, accept_len]) (lowest-index ties), never -1.
+ *   logits [S, K+1, V] float, draft [S, K] int32,
+ *   accept_len [S], next_token [S] int32 out.
+ *   Limits and errors as block_accept_greedy (K <= 32: at most 33 rows).
+ */
+int block_accept_greedy_bonus(const float *logits, const int32_t *draft, int S, int K,
+                              int V, int32_t *accept_len, int32_t *next_token,
+                              moe_stream_t stream);
+
+/*
+ * block_accept_rejection_bonus -- block_accept_rejection with a bonus row.
+ *   p holds K + 1 target rows per sequence, q the K draft rows.  Rows
+ *   0..K-1 are verified exactly as in block_accept_rejection (a rejection
+ *   at row a draws from max(0, p - q) at row a).  When all K drafts are
+ *   accepted the next token is drawn from the target row p[s, K] by the
+ *   same integer rule on P_v = floor(p_v * 2^40): m = floor(sum(P) * U /
+ *   2^24), U = u_resample[s] * 2^24, next_token = least v with
+ *   P_0 + .. + P_v > m.  A bonus row with no mass sets MOE_DEV_NO_MASS and
+ *   next_token = -1.
+ *   p [S, K+1, V], q [S, K, V] float; draft [S, K]; u_accept [S, K];
+ *   u_resample [S]; accept_len [S], next_token [S] int32 out.
+ *   Limits as block_accept_rejection.
+ */
+int block_accept_rejection_bonus(const float *p, const float *q, const int32_t *draft,
+                                 const float *u_accept, const float *u_resample,
+                                 int S, int K, int V, int32_t *accept_len,
+                                 int32_t *next_token, moe_stream_t stream);
+
+/*
+ * mxfp4_quantize -- bf16 weights to OCP MXFP4, the format the expert FFN
+ *   reads ([P3] "FP4 Expert 量化"; [P4] "第一层：FP4 选择性量化"; the
+ *   conversion is the one [OCP] defines).  Per 32 consecutive elements of
+ *   a row: scale byte e = max(0, floor(log2 amax) - 2 + 127) (byte 0 for an
+ *   all-zero block; bf16 inputs never need more than 252), and each element
+ *   becomes the E2M1 code nearest to v / 2^(e-127), ties to the even code,
+ *   saturating at +-6, with the sign of v (so -0 -> code 8).
+ *   w      [R, K] bf16, finite, 16-byte aligned
+ *   codes  [R, K/2] uint8 out (element 2j in the low nibble), 4-byte aligned
+ *   scales [R, K/32] uint8 out
+ *   Limits: K % 32 == 0, K >= 32, R >= 0, R * K <= 2^40.
+ *   Bound by HBM: 2 bytes read and 17/32 byte written per element.
+ */
+int mxfp4_quantize(const uint16_t *w, int64_t R, int K, uint8_t *codes, uint8_t *scales,
+                   moe_stream_t stream);
+
+/*
  * moe_get_device_status -- synchronise `stream`, then report the sticky
  * device status word of the current device: returns MOE_OK if it is clear,
  * MOE_ERR_DEVICE if set (detail in *detail, may be NULL), MOE_ERR_CUDA on a
@@ -283,6 +346,21 @@ int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
  */
 int moe_get_device_status(moe_stream_t stream, int *detail);
 int moe_clear_device_status(moe_stream_t stream);
+
+/*
+ * moe_set_wait_limit_ns -- time limit of the tensor-core FFN's bounded waits
+ *   on the current device: 2 s by default, `ns` = 0 restores the default.
+ *   (The pages have no counterpart; this is the library's failure
+ *   detection.)  A wait that runs past the limit ends the kernel early: it
+ *   sets MOE_DEV_TIMEOUT in the device status word, waits for the copies and
+ *   tensor-core operations it has already issued (at most 2 s more), frees
+ *   its tensor memory and returns, so the context stays usable and the next
+ *   call runs normally.  Lowering the limit far below a kernel's run time is
+ *   how that path is exercised; results of a call that timed out are
+ *   unspecified.  Enqueued on `stream` (the host value is copied before the
+ *   call returns).
+ */
+int moe_set_wait_limit_ns(uint64_t ns, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -43,8 +43,13 @@ SIGNATURES = {
     "block_accept_greedy": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "block_accept_rejection": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
                                         _vp, _vp, _vp]),
+    "block_accept_greedy_bonus": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "block_accept_rejection_bonus": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int,
+                                              _vp, _vp, _vp]),
+    "mxfp4_quantize": (_c_int, [_vp, ctypes.c_int64, _c_int, _vp, _vp, _vp]),
     "moe_get_device_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "moe_clear_device_status": (_c_int, [_vp]),
+    "moe_set_wait_limit_ns": (_c_int, [ctypes.c_uint64, _vp]),
 }
 
 _LIB = None
@@ -253,6 +258,58 @@ def block_accept_rejection(p, q, draft, u_accept, u_resample, accept_len=None,
     return accept_len, next_token
 
 
+def block_accept_greedy_bonus(logits, draft, accept_len=None, next_token=None, stream=None):
+    """logits [S, K+1, V] (row K: the target after the block), draft [S, K]."""
+    S, K1, V = logits.shape
+    K = K1 - 1
+    if tuple(draft.shape) != (S, K):
+        raise ValueError("draft must be [S, K] for logits [S, K+1, V]")
+    dev = logits.device
+    if accept_len is None:
+        accept_len = torch.empty(S, dtype=torch.int32, device=dev)
+    if next_token is None:
+        next_token = torch.empty(S, dtype=torch.int32, device=dev)
+    _check(lib().block_accept_greedy_bonus(_ptr(logits, torch.float32, "logits"),
+                                           _ptr(draft, torch.int32, "draft"), S, K, V,
+                                           _ptr(accept_len, torch.int32),
+                                           _ptr(next_token, torch.int32), _stream(stream)),
+           "block_accept_greedy_bonus")
+    return accept_len, next_token
+
+
+def block_accept_rejection_bonus(p, q, draft, u_accept, u_resample, accept_len=None,
+                                 next_token=None, stream=None):
+    """p [S, K+1, V] (row K: the target after the block), q [S, K, V]."""
+    S, K1, V = p.shape
+    K = K1 - 1
+    if tuple(q.shape) != (S, K, V) or tuple(draft.shape) != (S, K):
+        raise ValueError("q [S, K, V] and draft [S, K] for p [S, K+1, V]")
+    dev = p.device
+    if accept_len is None:
+        accept_len = torch.empty(S, dtype=torch.int32, device=dev)
+    if next_token is None:
+        next_token = torch.empty(S, dtype=torch.int32, device=dev)
+    _check(lib().block_accept_rejection_bonus(
+        _ptr(p, torch.float32, "p"), _ptr(q, torch.float32, "q"), _ptr(draft, torch.int32, "draft"),
+        _ptr(u_accept, torch.float32, "u_accept"), _ptr(u_resample, torch.float32, "u_resample"),
+        S, K, V, _ptr(accept_len, torch.int32), _ptr(next_token, torch.int32), _stream(stream)),
+        "block_accept_rejection_bonus")
+    return accept_len, next_token
+
+
+def mxfp4_quantize(w, codes=None, scales=None, stream=None):
+    """w [R, K] bf16 -> (codes [R, K/2] uint8, scales [R, K/32] uint8), OCP MXFP4."""
+    R, K = w.shape
+    dev = w.device
+    if codes is None:
+        codes = torch.empty((R, K // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((R, K // 32), dtype=torch.uint8, device=dev)
+    _check(lib().mxfp4_quantize(_ptr(w, torch.bfloat16, "w"), R, K, _ptr(codes, torch.uint8),
+                                _ptr(scales, torch.uint8), _stream(stream)), "mxfp4_quantize")
+    return codes, scales
+
+
 def moe_get_device_status(stream=None):
     """(status, detail): synchronises the stream and reads the status word."""
     d = ctypes.c_int(0)
@@ -262,3 +319,8 @@ def moe_get_device_status(stream=None):
 
 def moe_clear_device_status(stream=None):
     _check(lib().moe_clear_device_status(_stream(stream)), "moe_clear_device_status")
+
+
+def moe_set_wait_limit_ns(ns=0, stream=None):
+    """Limit of the FFN kernels' bounded waits (0 = the 2 s default)."""
+    _check(lib().moe_set_wait_limit_ns(int(ns), _stream(stream)), "moe_set_wait_limit_ns")

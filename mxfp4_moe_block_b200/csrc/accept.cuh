@@ -9,13 +9,20 @@
 // (i << 26 | argmax) to an atomicMin on the sequence's slot; the last of the
 // K rows to report turns the minimum into (accept_len, next_token).  The
 // slots are accept_len / next_token themselves, set up by a one-CTA kernel
-// launched just before.
+// launched just before.  With a bonus row (K+1 target rows per sequence, the
+// last one scoring the position after the block) that row has no draft and
+// always reports its argmax, so a sequence whose K drafts all match emits the
+// target's own next token (the target takes over after the last confirmed
+// token, "如何评价小米6月9日发布的MiMo-V2.5-Pro-UltraSpeed模式？", section
+// "二、投机解码").
 //
 // Rejection sampling ("MiMo-v2.5-Pro-UltraSpeed - infra 架构解读", section
 // "数据流概览"): exact test u*q(x) < p(x) in double, first rejection by
 // ballot, then an exact integer inverse-CDF draw from max(0, p - q): every
 // residual weight is an integer floor(r * 2^40), so the prefix sums are
-// independent of summation order and equal on every device.
+// independent of summation order and equal on every device.  With a bonus
+// row, a sequence whose K drafts are all accepted draws its next token from
+// the target row K by the same integer rule on floor(p * 2^40).
 #pragma once
 #include <cooperative_groups.h>
 #include "common.cuh"
@@ -54,11 +61,12 @@ greedy_init_kernel(int S, int32_t *__restrict__ accept_len, int32_t *__restrict_
   }
 }
 
-// grid (cluster_size, K, S), cluster (cluster_size, 1, 1), GREEDY_THREADS.
-// Rows hold finite values (a row of -inf reports token 0).
+// grid (cluster_size, R, S), cluster (cluster_size, 1, 1), GREEDY_THREADS;
+// R = K rows per sequence, or K + 1 with a bonus row.  Rows hold finite
+// values (a row of -inf reports token 0).
 __global__ void __launch_bounds__(GREEDY_THREADS)
 greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draft,
-              int S, int K, int V, int32_t *__restrict__ accept_len,
+              int S, int K, int V, int R, int32_t *__restrict__ accept_len,
               int32_t *__restrict__ next_token) {
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
@@ -73,7 +81,7 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
 
   // The logits were complete before the setup kernel passed its own wait,
   // so the scan needs no wait; only the slots do.
-  const float *row = logits + ((size_t)s * K + i) * V;
+  const float *row = logits + ((size_t)s * R + i) * V;
   float bv = -INFINITY;
   int bi = -1;
   if ((V & 3) == 0) {                  // rows 16-byte aligned: float4 units
@@ -124,15 +132,16 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
       if (better(pv, pi, v, m)) { v = pv; m = pi; }
     }
     m = max(m, 0);
-    const int d = __ldg(draft + (size_t)s * K + i);
-    if (d < 0 || d >= V) raise_status(MOE_DEV_BAD_TOKEN);
+    // the bonus row (i == K) has no draft: it always reports its argmax
+    const int d = i < K ? __ldg(draft + (size_t)s * K + i) : -1;
+    if (i < K && (d < 0 || d >= V)) raise_status(MOE_DEV_BAD_TOKEN);
     pdl_wait();                      // the slots were set up by greedy_init_kernel
     pdl_trigger();
     unsigned *key = reinterpret_cast<unsigned *>(accept_len + s);
     unsigned *cnt = reinterpret_cast<unsigned *>(next_token + s);
     if (d != m) atomicMin(key, ((unsigned)i << GREEDY_TOKEN_BITS) | (unsigned)m);
     __threadfence();
-    if (atomicAdd(cnt, 1u) == (unsigned)(K - 1)) {      // the last row of the sequence
+    if (atomicAdd(cnt, 1u) == (unsigned)(R - 1)) {      // the last row of the sequence
       __threadfence();
       const unsigned k = atomicOr(key, 0u);
       const bool miss = k != GREEDY_NO_MISS;
@@ -143,11 +152,12 @@ greedy_kernel(const float *__restrict__ logits, const int32_t *__restrict__ draf
   cluster.sync();   // keep every CTA's shared memory alive until CTA 0 is done
 }
 
-// One CTA per sequence.  blockDim.x is a multiple of 32, <= 1024.
+// One CTA per sequence.  blockDim.x is a multiple of 32, <= 1024.  p holds
+// R = K (+1 with a bonus row) rows per sequence, q holds K.
 __global__ void __launch_bounds__(1024)
 rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
                  const int32_t *__restrict__ draft, const float *__restrict__ u_accept,
-                 const float *__restrict__ u_resample, int S, int K, int V,
+                 const float *__restrict__ u_resample, int S, int K, int V, int R,
                  int32_t *__restrict__ accept_len, int32_t *__restrict__ next_token) {
   pdl_wait();
   pdl_trigger();
@@ -167,7 +177,8 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
         acc = false;
       } else {
         const double u = (double)__ldg(u_accept + row);
-        acc = u * (double)__ldg(q + row * V + x) < (double)__ldg(p + row * V + x);
+        const size_t prow = (size_t)s * R + lane;
+        acc = u * (double)__ldg(q + row * V + x) < (double)__ldg(p + prow * V + x);
       }
     }
     const unsigned rej = __ballot_sync(FULL, lane < K && !acc);
@@ -179,12 +190,15 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
   __syncthreads();
   const int a = s_a;
   if (tid == 0) accept_len[s] = a;
-  if (a == K) {
+  const bool bonus = R > K;
+  if (a == K && !bonus) {
     if (tid == 0) next_token[s] = -1;
     return;
   }
-  const float *pr = p + ((size_t)s * K + a) * V;
-  const float *qr = q + ((size_t)s * K + a) * V;
+  // row a of p (the bonus row K when every draft was accepted); q only
+  // below K
+  const float *pr = p + ((size_t)s * R + a) * V;
+  const float *qr = q + ((size_t)s * K + min(a, K - 1)) * V;
   const unsigned long long U = (unsigned long long)((double)__ldg(u_resample + s) * 16777216.0);
 
   // weight of token v: floor(max(0, p-q) * 2^40), or floor(p * 2^40) (mode 1)
@@ -205,7 +219,8 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
   };
 
   const int tile = blockDim.x;   // one element per thread per tile, coalesced
-  for (int mode = 0; mode < 2; ++mode) {
+  // the bonus draw takes p itself (mode 1) at once
+  for (int mode = a == K ? 1 : 0; mode < 2; ++mode) {
     unsigned long long mine = 0;
     for (int v = tid; v < V; v += tile) mine += weight(v, mode);
     const unsigned long long total = block_sum(mine);

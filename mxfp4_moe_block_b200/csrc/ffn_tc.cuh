@@ -30,6 +30,7 @@
 // drains what it issued, frees its TMEM and returns.
 #pragma once
 #include <cuda.h>
+#include <mutex>
 #include "common.cuh"
 #include "ffn_fma.cuh"
 
@@ -73,20 +74,40 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Bounded wait: false (and the status word set) after ~2 s.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Bounded waits.  The pipeline's waits give up after g_wait_limit_ns (2 s
+// unless moe_set_wait_limit_ns lowered it): the waiting role sets the CTA's
+// abort flag and the status word (MOE_DEV_TIMEOUT), and every role then
+// leaves its loop.  The drain at the end of the kernel -- for copies and MMAs
+// already issued -- has its own fixed limit, so that a lowered pipeline limit
+// never cuts a drain short.
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
 __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
+  const uint64_t limit = *(volatile unsigned long long *)&g_wait_limit_ns;
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 63) {
       if (*abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 >= limit) {
         raise_status(MOE_DEV_TIMEOUT);
         *abort = 1;
         return false;
       }
+    }
+  }
+}
+
+// Wait for the completion of work already issued (abort flag ignored).
+__device__ __noinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && global_ns() - t0 >= kDrainLimitNs) {
+      raise_status(MOE_DEV_TIMEOUT);
+      return false;
     }
   }
 }
@@ -220,6 +241,25 @@ __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sy
 __device__ __forceinline__ void group_sync(int grp) {
   if (grp) asm volatile("bar.sync 2, 128;" ::: "memory");
   else asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// The same barrier, returning true iff `v` holds on every thread of the
+// group: the group's warps take each leave-or-stay decision together, so no
+// warp can wait at group_sync for one that has left.
+__device__ __forceinline__ bool group_all(int grp, bool v) {
+  uint32_t r;
+  __syncwarp();
+  if (grp)
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v) : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)v) : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -599,6 +639,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   uint64_t *ring_full = sfs_full + C::kStages;  // [kRing]
   uint64_t *ring_empty = ring_full + kRing;     // [kRing]
   volatile int *ring = reinterpret_cast<volatile int *>(ring_empty + kRing);   // [kRing]
+  // end of the kernel: the MMA thread's last commit, and the number of
+  // stages the producer issued (the abort path drains them)
+  uint64_t *drain_bar = ring_empty + kRing + 2;
+  volatile int *s_issued = reinterpret_cast<volatile int *>(drain_bar + 1);
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
   // The table stays small: a GEMM CTA leaves a few KB of the SM's shared
   // memory free, so that the encode kernels' CTAs can become resident beside
@@ -655,7 +699,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4 * Kd::kEpiGroups);   // one arrival per epilogue warp
     }
+    mbar_init(drain_bar, 1);           // the MMA thread's final commit
     *abort = 0;
+    *s_issued = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   } else if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -696,6 +742,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     nB = min(BN, T * ne - nt * BN);
   };
 
+  int w_arrived = 0;   // stages an A-scale writer warp has released (abort drain)
+  int l_signaled = 0;  // stages the scale loader has signalled (abort drain)
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer --
     if (lane == 0) {
@@ -776,14 +824,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         t = t_next;
       }
       if (*abort) publish(n_tiles);            // release readers still waiting
-      // drain: wait (bounded) until the last issued stages have landed
-      if (*abort) {
-        for (int s = 0; s < C::kStages && s < issued; ++s) {
-          if (--stage < 0) { stage = C::kStages - 1; phase ^= 1; }
-          volatile int never = 0;
-          mbar_wait(&full[stage], phase, (volatile int *)&never);
-        }
-      }
+      *s_issued = issued;                      // read after the role loops end
     }
   } else if (warp == 1) {
     // --------------------------------------------------- scale loader --
@@ -792,12 +833,14 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     // byte 16*(row%32) + 4*(row/32) + (k-block within the group).
     const uint32_t kb = a.K / 32;            // scale bytes per row
     if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
+    // Leave-or-stay decisions are warp-wide, so that every stage this warp
+    // signals gets all 32 lanes' arrivals.
     int stage = 0;
     uint32_t phase = 0;
-    int ti = 0;
-    for (int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
-         t < n_tiles && !*abort;
-         t = ring_read(ring_full, ring_empty, ring, ++ti, lane == 0, abort, n_tiles)) {
+    bool ok = true;
+    for (int ti = 0; ok; ++ti) {
+      const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+      if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
       int e, mt, rowB, nB;
       decode(t, e, mt, rowB, nB);
       const int ebase = e * a.rows_per_expert;
@@ -811,7 +854,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         src_a[q] = a.a_scales + (size_t)row * kb;
       }
       for (int kt = 0; kt < ksteps; ++kt) {
-        if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
+        if (!__all_sync(FULL, mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
+          ok = false;
+          break;
+        }
         uint8_t *sfa = smem + C::kOffSfa + stage * C::kSfa;
         uint8_t *sfb = smem + C::kOffSfb + stage * C::kSfb;
 #pragma unroll
@@ -829,6 +875,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           }
         }
         cp_async_arrive_noinc(&sfs_full[stage]);
+        ++l_signaled;
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -919,6 +966,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         if (!ok) break;
         tc_commit(&acc_full[buf]);
       }
+      // Every MMA and tensor-memory copy this thread issued completes before
+      // the CTA frees its tensor memory, on every exit path: one more commit
+      // tracks them all.  (On the normal path the epilogue has waited for the
+      // last tile already, so this costs nothing.)
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0);
     }
   } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------- A-scale writers --
@@ -927,19 +980,22 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     // four quarters), keeping the copies off the MMA issue path.  Column
     // 4g + j, lane l = the 4 scale bytes of tile row 32j + l, K-group g: the
     // 16 bytes the scale loader put at 512g + 16l.
+    // Each leave-or-stay decision is taken by the whole warp (__all_sync):
+    // tcgen05.st and tcgen05.wait::st need all 32 lanes.
     const int q = warp - 8;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int stage = 0;
     uint32_t phase = 0;
-    int ti = 0;
-    for (int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
-         t < n_tiles && !*abort;
-         t = ring_read(ring_full, ring_empty, ring, ++ti, lane == 0, abort, n_tiles)) {
+    bool ok = true;
+    for (int ti = 0; ok; ++ti) {
+      const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+      if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
       for (int kt = 0; kt < ksteps; ++kt) {
         // the MMAs that read this stage's columns last time are done, and the
         // stage's scale bytes are in shared memory
-        if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
-        if (!mbar_wait_fast(&sfs_full[stage], phase, abort)) break;
+        const bool ready = mbar_wait_fast(&empty[stage], phase ^ 1, abort) &&
+                           mbar_wait_fast(&sfs_full[stage], phase, abort);
+        if (!__all_sync(FULL, ready)) { ok = false; break; }
         tc_fence_after();
         const uint4 *src =
             reinterpret_cast<const uint4 *>(smem + C::kOffSfa + stage * C::kSfa) + lane;
@@ -957,6 +1013,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&full[stage]);
+        ++w_arrived;
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -971,27 +1028,31 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     float *gx = xchg + grp * C::kXchgFloats;
     pdl_wait();                                 // row scales in, h / y out
     constexpr int kTokPerLd = 16 / T;           // tokens per 16-column load
-    int it = 0;
-    for (int t = ring_read(ring_full, ring_empty, ring, it, lane == 0, abort, n_tiles);
-         t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, lane == 0, abort, n_tiles)) {
-      int e, mt, rowB, nB;
-      decode(t, e, mt, rowB, nB);
+    for (int it = 0;; ++it) {
+      const int t = ring_read(ring_full, ring_empty, ring, it, lane == 0, abort, n_tiles);
+      bool ok = t < n_tiles && !*abort;
+      int e = 0, mt = 0, rowB = 0, nB = 0;
+      if (ok) decode(t, e, mt, rowB, nB);
       const int buf = it % C::kAcc;
       const uint32_t use = (uint32_t)(it / C::kAcc);
-      const int ntok = nB / T;                  // tokens in this tile
+      const int ntok = nB / T;                  // tokens in this tile (>= 1 in a tile)
       const int rtok0 = rowB / T;               // sorted row of the tile's first token
       // the first chunk's row scales do not depend on the accumulator: load
       // them while the MMAs still run
       const int cfirst = 16 * grp;              // this group's first chunk
       float rs0[16];
       if (Kd::kRowScaledB) {
+        // (rows past ntok are discarded; with no tile the index stays at 0)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int tok = min((cfirst + i) / T, ntok - 1);   // rows past ntok are discarded
+          const int tok = max(0, min((cfirst + i) / T, ntok - 1));
           rs0[i] = __ldg(a.b_rowscale + (size_t)(rtok0 + tok) * T + i % T);
         }
       }
-      if (!mbar_wait_fast(&acc_full[buf], use & 1, abort)) break;
+      if (ok) ok = mbar_wait_fast(&acc_full[buf], use & 1, abort);
+      // the group's four warps leave together: at the end of the tiles, or
+      // when any of them saw the abort flag or a wait run out
+      if (!group_all(grp, ok)) break;
       tc_fence_after();
       const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
       if (cfirst >= nB) {
@@ -1084,7 +1145,28 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     }
   }
 
+  // Every role has left its loop, and the MMA thread's issued work is
+  // complete.  After an abort, TMA loads may still be in flight into stages
+  // the MMA never consumed: the A-scale writers make the arrivals they owe on
+  // those stages' full barriers (the producer issued at most kStages ahead of
+  // them), so that each barrier's phase now waits for its TMA bytes alone,
+  // and the producer waits (bounded) for the last stages it issued to land
+  // before the CTA's shared memory is released.
   __syncthreads();
+  if (*abort) {
+    const int issued = *s_issued;
+    if (warp >= 8 && warp < 12 && lane == 0)
+      for (int j = w_arrived; j < issued; ++j) mbar_arrive(&full[j % C::kStages]);
+    __syncthreads();
+    if (warp == 0 && lane == 0)
+      for (int j = max(0, issued - C::kStages); j < issued; ++j)
+        mbar_wait_drain(&full[j % C::kStages], (uint32_t)(j / C::kStages) & 1u);
+    // the scale loader's last signals: their cp.async arrivals have landed
+    if (warp == 1)
+      for (int j = max(0, l_signaled - C::kStages); j < l_signaled; ++j)
+        mbar_wait_drain(&sfs_full[j % C::kStages], (uint32_t)(j / C::kStages) & 1u);
+    __syncthreads();
+  }
   if (warp == 2) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -1127,18 +1209,20 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once per process (a function-
+// local static: its initialisation is thread-safe).
 inline EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return (EncodeTiledFn) nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
   return fn;
 }
 
@@ -1166,6 +1250,76 @@ inline bool make_weight_map(CUtensorMap *m, const uint8_t *codes, uint64_t K, ui
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, codes, K, rows, K / 2, 128, 64);
 }
 
+// Maximum dynamic shared memory of the two GEMM kernels of one
+// instantiation, set once per device; a failed set is reported and retried
+// on the next call.  Guarded by a mutex: host threads may make their first
+// call at the same time.
+template <int KIND, int BN>
+inline int tc_attributes(int dev) {
+  using C = TcCfg<KIND, BN>;
+  static std::mutex mu;
+  static unsigned long long done = 0;   // one bit per device
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if ((done >> dev) & 1ull) return MOE_OK;
+  if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, 1, BN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(tc_gemm_kernel<KIND, 2, BN>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  done |= 1ull << dev;
+  return MOE_OK;
+}
+
+// The tensor maps of one FFN call depend only on its pointers and sizes;
+// callers that run the same problem again (an eager decode loop) find them
+// here instead of encoding twelve maps on the host per call.  A handful of
+// entries, replaced round-robin, under a mutex.
+struct TcMapKey {
+  int kind, bn, dev, H, I, E;
+  size_t P;
+  const void *w13c, *w2c, *xq, *hq;
+  bool operator==(const TcMapKey &o) const {
+    return kind == o.kind && bn == o.bn && dev == o.dev && H == o.H && I == o.I && E == o.E &&
+           P == o.P && w13c == o.w13c && w2c == o.w2c && xq == o.xq && hq == o.hq;
+  }
+};
+
+struct TcMapCache {
+  static constexpr int kEntries = 8;
+  std::mutex mu;
+  TcMapKey key[kEntries];
+  TcMaps m1[kEntries], m2[kEntries];
+  bool used[kEntries] = {};
+  int next = 0;
+  bool find(const TcMapKey &k, TcMaps &a, TcMaps &b) {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < kEntries; ++i)
+      if (used[i] && key[i] == k) {
+        a = m1[i];
+        b = m2[i];
+        return true;
+      }
+    return false;
+  }
+  void put(const TcMapKey &k, const TcMaps &a, const TcMaps &b) {
+    std::lock_guard<std::mutex> lk(mu);
+    const int i = next;
+    next = (next + 1) % kEntries;
+    key[i] = k;
+    m1[i] = a;
+    m2[i] = b;
+    used[i] = true;
+  }
+};
+
+inline TcMapCache &tc_map_cache() {
+  static TcMapCache c;
+  return c;
+}
+
 template <int KIND, int BN>
 int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   using C = TcCfg<KIND, BN>;
@@ -1182,15 +1336,42 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   int *counters = reinterpret_cast<int *>(hs + align256_tc(tc_scale_bytes(P, I)));
 
   int dev = 0;
-  cudaGetDevice(&dev);
-  static unsigned long long attr_done = 0;      // one bit per device
-  if (dev < 64 && !((attr_done >> dev) & 1ull)) {
-    attr_done |= 1ull << dev;
-    cudaFuncSetAttribute(tc_gemm_kernel<KIND, 1, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         C::kSmem);
-    cudaFuncSetAttribute(tc_gemm_kernel<KIND, 2, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         C::kSmem);
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
+  const int st = tc_attributes<KIND, BN>(dev);
+  if (st != MOE_OK) return st;
+
+  TcArgs a{};
+  a.off = f.off;
+  a.E = E;
+  a.P = (int)P;
+  a.I = I;
+  a.H = H;
+  a.h = f.h;
+  a.hq = hq;
+  a.hs = hs;
+  a.y = f.y;
+  for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
+
+  // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]; GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
+  TcMaps maps1, maps2;
+  const TcMapKey key{KIND, BN, dev, H, I, E, P, f.w13c, f.w2c, xq, hq};
+  if (!tc_map_cache().find(key, maps1, maps2)) {
+    if (!make_weight_map<KIND>(&maps1.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
+    for (int i = 0; i < 5; ++i)
+      if (!make_map(&maps1.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
+                    a.b_box[i]))
+        return MOE_ERR_CUDA;
+    if (!make_weight_map<KIND>(&maps2.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
+    for (int i = 0; i < 5; ++i)
+      if (!make_map(&maps2.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
+                    a.b_box[i]))
+        return MOE_ERR_CUDA;
+    tc_map_cache().put(key, maps1, maps2);
+  }
+
   if (KIND == KIND_F4) {
     if (launch_encode_f4<T>(f.x, f.sp, f.k, H, P, xq, reinterpret_cast<float *>(xs), 0, counters,
                             s) != cudaSuccess)
@@ -1202,43 +1383,20 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
         cudaSuccess)
       return MOE_ERR_CUDA;
   }
-  TcMaps maps;
-  TcArgs a{};
-  a.off = f.off;
-  a.E = E;
-  a.P = (int)P;
-  a.I = I;
-  a.H = H;
-  a.h = f.h;
-  a.hq = hq;
-  a.hs = hs;
-  a.y = f.y;
-  a.tile_counter = counters;
-  for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
 
-  // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]
-  if (!make_weight_map<KIND>(&maps.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
-  for (int i = 0; i < 5; ++i)
-    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
-                  a.b_box[i]))
-      return MOE_ERR_CUDA;
   a.a_scales = f.w13s;
   a.b_scales = xs;
   a.b_rowscale = reinterpret_cast<const float *>(xs);
   a.K = H;
   a.rows_per_expert = 2 * I;
-  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps, a) != cudaSuccess)
+  a.tile_counter = counters;
+  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
 
   if (KIND == KIND_F4)
     if (launch_encode_f4<T>(f.h, nullptr, 1, I, P, hq, reinterpret_cast<float *>(hs), 1, nullptr,
                             s) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  // GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
-  if (!make_weight_map<KIND>(&maps.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
-  for (int i = 0; i < 5; ++i)
-    if (!make_map(&maps.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
-                  a.b_box[i]))
       return MOE_ERR_CUDA;
   a.a_scales = f.w2s;
   a.b_scales = hs;
@@ -1246,7 +1404,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.K = I;
   a.rows_per_expert = H;
   a.tile_counter = counters + 1;
-  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, Kd::kThreads, C::kSmem, s, maps, a) != cudaSuccess)
+  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, Kd::kThreads, C::kSmem, s, maps2, a) !=
+      cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

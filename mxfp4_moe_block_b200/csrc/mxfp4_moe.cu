@@ -12,6 +12,7 @@
 #include "ffn_tc.cuh"
 #include "combine.cuh"
 #include "accept.cuh"
+#include "quantize.cuh"
 
 using namespace moe;
 
@@ -274,7 +275,11 @@ int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
                           const uint8_t *w2_codes, const uint8_t *w2_scales,
                           const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
                           moe_stream_t stream) {
-  if (T < 0 || k < 1 || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+  // the argument checks of mxfp4_moe_ffn_variant first, so that a bad
+  // argument is reported as such whatever the problem's scratch need
+  if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
+  if (H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
+  if (E > 1024) return MOE_ERR_UNSUPPORTED;
   if (mxfp4_moe_ffn_workspace_bytes(T, k, H, I) > (size_t)MOE_NOALLOC_SCRATCH_BYTES) {
     fprintf(stderr,
             "mxfp4_moe_ffn_noalloc: T=%d k=%d H=%d I=%d needs %zu scratch bytes, more than the "
@@ -324,8 +329,10 @@ int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
 }
 
 // ----------------------------------------------------------------- accept --
-int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K, int V,
-                        int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+// Greedy acceptance over R target rows per sequence (R = K, or K + 1 with a
+// bonus row).
+static int greedy_launch(const float *logits, const int32_t *draft, int S, int K, int V, int R,
+                         int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
   if (S < 0 || K < 1 || K > 32 || V < 1) return MOE_ERR_INVALID_ARG;
   if (S == 0) return MOE_OK;
   if (!logits || !draft || !accept_len || !next_token) return MOE_ERR_INVALID_ARG;
@@ -344,7 +351,7 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
   const cudaStream_t s = (cudaStream_t)stream;
   // Cluster size per row: slices of about 48 KB, at least two CTAs per SM
   // over all rows, at least GREEDY_THREADS elements (or float4 units) each.
-  const long long rows = (long long)S * K;
+  const long long rows = (long long)S * R;
   const long long units = (V & 3) == 0 ? V / 4 : V;
   long long csize = std::max<long long>((4LL * V + 49151) / 49152, (2LL * dev->sms + rows - 1) / rows);
   csize = std::min<long long>(csize, std::max<long long>(1, units / GREEDY_THREADS));
@@ -354,7 +361,7 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
                                256, 0, s, S, accept_len, next_token));
   if (st != MOE_OK) return st;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)csize, (unsigned)K, (unsigned)S);
+  cfg.gridDim = dim3((unsigned)csize, (unsigned)R, (unsigned)S);
   cfg.blockDim = dim3(GREEDY_THREADS, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
@@ -368,12 +375,22 @@ int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K,
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return launched(
-      cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, accept_len, next_token));
+      cudaLaunchKernelEx(&cfg, greedy_kernel, logits, draft, S, K, V, R, accept_len, next_token));
 }
 
-int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
-                           const float *u_accept, const float *u_resample, int S, int K, int V,
-                           int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K, int V,
+                        int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  return greedy_launch(logits, draft, S, K, V, K, accept_len, next_token, stream);
+}
+
+int block_accept_greedy_bonus(const float *logits, const int32_t *draft, int S, int K, int V,
+                              int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  return greedy_launch(logits, draft, S, K, V, K + 1, accept_len, next_token, stream);
+}
+
+static int rejection_launch(const float *p, const float *q, const int32_t *draft,
+                            const float *u_accept, const float *u_resample, int S, int K, int V,
+                            int R, int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
   if (S < 0 || K < 1 || K > 32 || V < 1 || V > (1 << 24)) return MOE_ERR_INVALID_ARG;
   if (S == 0) return MOE_OK;
   if (!p || !q || !draft || !u_accept || !u_resample || !accept_len || !next_token)
@@ -382,7 +399,40 @@ int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
   int threads = ((V + 31) / 32) * 32;
   if (threads > 1024) threads = 1024;
   return launched(launch_pdl(rejection_kernel, S, threads, 0, (cudaStream_t)stream, p, q, draft,
-                             u_accept, u_resample, S, K, V, accept_len, next_token));
+                             u_accept, u_resample, S, K, V, R, accept_len, next_token));
+}
+
+int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
+                           const float *u_accept, const float *u_resample, int S, int K, int V,
+                           int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  return rejection_launch(p, q, draft, u_accept, u_resample, S, K, V, K, accept_len, next_token,
+                          stream);
+}
+
+int block_accept_rejection_bonus(const float *p, const float *q, const int32_t *draft,
+                                 const float *u_accept, const float *u_resample, int S, int K,
+                                 int V, int32_t *accept_len, int32_t *next_token,
+                                 moe_stream_t stream) {
+  return rejection_launch(p, q, draft, u_accept, u_resample, S, K, V, K + 1, accept_len,
+                          next_token, stream);
+}
+
+// --------------------------------------------------------------- quantise --
+int mxfp4_quantize(const uint16_t *w, int64_t R, int K, uint8_t *codes, uint8_t *scales,
+                   moe_stream_t stream) {
+  if (R < 0 || K < 32 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (R == 0) return MOE_OK;
+  if (!w || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(w) & 15) || (reinterpret_cast<uintptr_t>(codes) & 3))
+    return MOE_ERR_INVALID_ARG;
+  if (R > (int64_t(1) << 40) / K) return MOE_ERR_UNSUPPORTED;
+  const DeviceInfo *dev = device_info();
+  if (!dev) return MOE_ERR_CUDA;
+  const size_t n8 = (size_t)R * (size_t)K / 8;
+  const size_t blocks = (n8 + QUANT_THREADS - 1) / QUANT_THREADS;
+  const unsigned grid = (unsigned)std::min<size_t>(blocks, (size_t)dev->sms * 8);
+  return launched(launch_pdl(mxfp4_quantize_kernel, grid, QUANT_THREADS, 0, (cudaStream_t)stream,
+                             w, n8, codes, scales));
 }
 
 // ----------------------------------------------------------------- status --
@@ -392,6 +442,17 @@ int moe_get_device_status(moe_stream_t stream, int *detail) {
   if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
   if (detail) *detail = v;
   return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+int moe_set_wait_limit_ns(uint64_t ns, moe_stream_t stream) {
+  // the host value is staged by the runtime before the call returns
+  const unsigned long long v = ns ? (unsigned long long)ns : 2000000000ull;
+  if (cudaMemcpyToSymbolAsync(g_wait_limit_ns, &v, sizeof(v), 0, cudaMemcpyHostToDevice,
+                              (cudaStream_t)stream) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 
 int moe_clear_device_status(moe_stream_t stream) {

@@ -1,0 +1,79 @@
+// quantize.cuh -- bf16 weights -> OCP MXFP4 (E2M1 codes + E8M0 block scales).
+//
+// The expert weights the verify step streams are MXFP4 ("MiMo-v2.5-Pro-
+// UltraSpeed - infra 架构解读", section "FP4 Expert 量化";
+// "mimo-tilert-1000tps-trillion-parameter-inference", section "第一层：FP4
+// 选择性量化").  This kernel produces that format from bf16 weights by the
+// OCP MX v1.0 conversion: per 32 consecutive elements of a row the shared
+// scale is 2^(floor(log2 amax) - 2) (2 = the largest E2M1 exponent), and each
+// element becomes the nearest E2M1 value of v / scale, ties to the even
+// code, saturating at +-6, its sign kept.
+//
+// HBM-bound: 2 bytes read and 17/32 byte written per element.  Each thread
+// takes 8 consecutive elements (one 16-byte load, one 4-byte store of codes);
+// four neighbouring threads hold a 32-element block and meet by shuffles.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int QUANT_THREADS = 256;
+
+// E2M1 magnitude index (0..7 for 0, .5, 1, 1.5, 2, 3, 4, 6) nearest to a >= 0,
+// ties to the even index, a > 6 saturating at 7.  The midpoints between
+// neighbours are .25 .75 1.25 1.75 2.5 3.5 5; at a midpoint the comparison
+// is strict where the lower neighbour is even and inclusive where the upper
+// one is.
+__device__ __forceinline__ uint32_t e2m1_nearest_even(float a) {
+  return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+         (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
+         (uint32_t)(a > 5.0f);
+}
+
+// w: n8 groups of 8 bf16 (n8 = R*K/8); codes: 4 bytes per group; scales: one
+// byte per 4 groups.
+__global__ void __launch_bounds__(QUANT_THREADS)
+mxfp4_quantize_kernel(const uint16_t *__restrict__ w, size_t n8, uint8_t *__restrict__ codes,
+                      uint8_t *__restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const unsigned lane = threadIdx.x & 31;
+  // the loop bound is warp-uniform (every lane takes part in the shuffles);
+  // n8 is a multiple of 4, so the four threads of a block are valid together
+  for (size_t g0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x - lane; g0 < n8; g0 += stride) {
+    const size_t g = g0 + lane;
+    const bool valid = g < n8;
+    const uint4 v = valid ? ld_stream16(w + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    // largest magnitude of the block: bf16 bit patterns without the sign
+    // compare like the magnitudes they encode
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, max(wd[i] & 0x7fffu, (wd[i] >> 16) & 0x7fffu));
+    m = max(m, __shfl_xor_sync(FULL, m, 1));
+    m = max(m, __shfl_xor_sync(FULL, m, 2));
+    // scale byte = floor(log2 amax) - 2 + 127 = (biased exponent of amax) - 2,
+    // at least 0 (all-zero and tiny blocks); bf16 exponents stop at 254, so
+    // the byte never exceeds 252
+    const int be = (int)(m >> 7);
+    const uint32_t sb = (uint32_t)max(0, be - 2);
+    const float inv = __uint_as_float((254u - sb) << 23);   // 2^(127 - sb), exact
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t b = (i & 1) ? (wd[i >> 1] >> 16) : (wd[i >> 1] & 0xffffu);
+      // |v| * 2^(127 - sb) is exact wherever it can reach 0.25 (no overflow:
+      // it stays below 8)
+      const float a = __uint_as_float((b & 0x7fffu) << 16) * inv;
+      const uint32_t c = e2m1_nearest_even(a) | ((b >> 12) & 8u);   // sign -> bit 3
+      word |= c << (4 * i);
+    }
+    if (valid) {
+      *reinterpret_cast<uint32_t *>(codes + 4 * g) = word;
+      if ((g & 3) == 0) scales[g >> 2] = (uint8_t)sb;
+    }
+  }
+}
+
+}  // namespace moe

@@ -284,13 +284,27 @@ def _target_argmax(logits: np.ndarray) -> np.ndarray:
     return np.argmax(logits, axis=-1)
 
 
-def block_logits(sh: Shape, layer: int = 0) -> np.ndarray:
-    """Target logits [S, K, V] float32: N(0, 2) (2 = standard deviation)."""
-    z = normal_np(stream_key(sh.seed, "block_logits", layer), 0, sh.S * sh.K * sh.V)
-    return (2.0 * z).astype(np.float32).reshape(sh.S, sh.K, sh.V)
+def _seq_range(sh: Shape, seqs) -> tuple:
+    s0, s1 = (0, sh.S) if seqs is None else seqs
+    if not 0 <= s0 < s1 <= sh.S:
+        raise ValueError("sequence range outside [0, S)")
+    return s0, s1
 
 
-def greedy_drafts(sh: Shape, logits: np.ndarray, rule: str | None = None) -> np.ndarray:
+def block_logits(sh: Shape, layer: int = 0, rows: int | None = None, seqs=None) -> np.ndarray:
+    """Target logits [S, R, V] float32: N(0, 2) (2 = standard deviation).
+
+    R = K by default; R = K + 1 draws blocks with a bonus row (the target's
+    scores for the position after the block).  ``seqs`` = (s0, s1) draws
+    only those sequences (the same values as rows s0..s1-1 of the full draw)."""
+    R = sh.K if rows is None else rows
+    s0, s1 = _seq_range(sh, seqs)
+    z = normal_np(stream_key(sh.seed, "block_logits", layer), s0 * R * sh.V, (s1 - s0) * R * sh.V)
+    return (2.0 * z).astype(np.float32).reshape(s1 - s0, R, sh.V)
+
+
+def greedy_drafts(sh: Shape, logits: np.ndarray, rule: str | None = None,
+                  seqs=None) -> np.ndarray:
     """Draft tokens [S, K] int32 built around the target argmax.
 
     'perturb4'  : each position independently replaced w.p. 1/4 by
@@ -300,18 +314,20 @@ def greedy_drafts(sh: Shape, logits: np.ndarray, rule: str | None = None) -> np.
                   above, later positions are uniform over the vocabulary.
     """
     rule = rule or sh.draft_rule
-    S, K, V = sh.S, sh.K, sh.V
+    K, V = sh.K, sh.V
+    s0, s1 = _seq_range(sh, seqs)
+    S = s1 - s0
     am = _target_argmax(logits).astype(np.int64)
-    r = int_range_np(stream_key(sh.seed, "draft_perturb"), 0, S * K, 0, V - 2).reshape(S, K)
+    r = int_range_np(stream_key(sh.seed, "draft_perturb"), s0 * K, S * K, 0, V - 2).reshape(S, K)
     pert = (am + 1 + r) % V
     if rule == "perturb4":
-        pick = int_range_np(stream_key(sh.seed, "draft_pos"), 0, S * K, 0, 3).reshape(S, K) == 0
+        pick = int_range_np(stream_key(sh.seed, "draft_pos"), s0 * K, S * K, 0, 3).reshape(S, K) == 0
         d = np.where(pick, pert, am)
     else:
-        u = u53_np(stream_key(sh.seed, "geom"), 0, S)
+        u = u53_np(stream_key(sh.seed, "geom"), s0, S)
         # inverse CDF of Geometric(p) on {0,1,...}: floor(log(1-u)/log(1-p))
         L = np.floor(np.log1p(-u) / math.log1p(-1.0 / 7.0)).astype(np.int64)
-        rnd = int_range_np(stream_key(sh.seed, "draft_random"), 0, S * K, 0, V - 1).reshape(S, K)
+        rnd = int_range_np(stream_key(sh.seed, "draft_random"), s0 * K, S * K, 0, V - 1).reshape(S, K)
         pos = np.arange(K)[None, :]
         d = np.where(pos < L[:, None], am, np.where(pos == L[:, None], pert, rnd))
     return d.astype(np.int32)
@@ -332,17 +348,27 @@ class RejectionInputs:
     u_resample: np.ndarray # [S] float32 (multiples of 2**-24)
 
 
-def rejection_inputs(sh: Shape, layer: int = 0) -> RejectionInputs:
-    """p, q = softmax of independent N(0,2) logits; drafts x_i ~ q_i."""
-    S, K, V = sh.S, sh.K, sh.V
+def rejection_inputs(sh: Shape, layer: int = 0, bonus: bool = False,
+                     seqs=None) -> RejectionInputs:
+    """p, q = softmax of independent N(0,2) logits; drafts x_i ~ q_i.
+
+    With ``bonus`` p has K + 1 rows per sequence (row K: the target after the
+    block); q and the drafts keep K.  ``seqs`` = (s0, s1) draws only those
+    sequences (the same values as rows s0..s1-1 of the full draw)."""
+    K, V = sh.K, sh.V
+    s0, s1 = _seq_range(sh, seqs)
+    S = s1 - s0
     n = S * K * V
-    zp = 2.0 * normal_np(stream_key(sh.seed, "p_logits", layer), 0, n).reshape(S, K, V)
-    zq = 2.0 * normal_np(stream_key(sh.seed, "q_logits", layer), 0, n).reshape(S, K, V)
+    Kp = K + 1 if bonus else K
+    zp = 2.0 * normal_np(stream_key(sh.seed, "p_logits", layer), s0 * Kp * V,
+                         S * Kp * V).reshape(S, Kp, V)
+    zq = 2.0 * normal_np(stream_key(sh.seed, "q_logits", layer), s0 * K * V, n).reshape(S, K, V)
     p = _softmax64(zp).astype(np.float32)
     q = _softmax64(zq).astype(np.float32)
-    draft = sample_rows_np(q, u53_np(stream_key(sh.seed, "u_draft", layer), 0, S * K).reshape(S, K))
-    ua = u24_np(stream_key(sh.seed, "u_accept", layer), 0, S * K).reshape(S, K)
-    ur = u24_np(stream_key(sh.seed, "u_resample", layer), 0, S)
+    draft = sample_rows_np(q, u53_np(stream_key(sh.seed, "u_draft", layer), s0 * K,
+                                     S * K).reshape(S, K))
+    ua = u24_np(stream_key(sh.seed, "u_accept", layer), s0 * K, S * K).reshape(S, K)
+    ur = u24_np(stream_key(sh.seed, "u_resample", layer), s0, S)
     return RejectionInputs(p, q, draft, ua, ur)
 
 

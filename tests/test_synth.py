@@ -77,3 +77,24 @@ def test_drafts_follow_rules():
     prefix = np.where(match.all(1), sh2.K, np.argmin(match, 1))
     # Geometric(1/7) prefix truncated at K = 8: mean = 6 * (1 - (6/7)**8)
     assert abs(prefix.mean() - 6 * (1 - (6 / 7) ** 8)) < 0.15
+
+
+def test_sequence_range_draws_equal_rows_of_the_full_draw():
+    """Drawing only sequences s0..s1-1 (the oracle's bounded samples do) gives
+    the same values as those rows of the full draw, for every recipe."""
+    sh = synth.Shape("t", H=256, I=128, E=8, k=2, S=5, K=4, V=300, seed=9)
+    full = synth.block_logits(sh)
+    part = synth.block_logits(sh, seqs=(2, 4))
+    assert np.array_equal(full[2:4], part)
+    for rule in ("geometric", "perturb4"):
+        assert np.array_equal(synth.greedy_drafts(sh, full, rule)[2:4],
+                              synth.greedy_drafts(sh, part, rule, seqs=(2, 4)))
+    for bonus in (False, True):
+        r = synth.rejection_inputs(sh, bonus=bonus)
+        rp = synth.rejection_inputs(sh, bonus=bonus, seqs=(1, 3))
+        for a, b in zip((r.p, r.q, r.draft, r.u_accept, r.u_resample),
+                        (rp.p, rp.q, rp.draft, rp.u_accept, rp.u_resample)):
+            assert np.array_equal(a[1:3], b)
+    lb = synth.block_logits(sh, rows=sh.K + 1)
+    assert lb.shape == (sh.S, sh.K + 1, sh.V)
+    assert np.array_equal(lb[3:5], synth.block_logits(sh, rows=sh.K + 1, seqs=(3, 5)))

@@ -172,6 +172,17 @@ enum {
                             activation terms with one scale per row and term
                             (H, I multiples of 256, at most 8192)                 */
 };
+/* Accuracy domain of the activation encodings.  FMA and TENSOR_F8 represent
+ * every 32-element block of an activation row on its own scale, so they meet
+ * the FFN tolerance for any finite bf16 rows and any weights whose values are
+ * finite bf16 numbers.  TENSOR_F4 (which TENSOR and AUTO take for narrow
+ * tiles) represents a whole row by eight terms, each element exact to about
+ * 2^-16 of the row's largest magnitude; that meets the tolerance unless the
+ * products of a row's 32-element blocks with their weight blocks span more
+ * than about 2^16 -- small activation blocks meeting weight scales 2^16 times
+ * larger than those of the row's large blocks.  Such weights (E8M0 scales
+ * spread over more than 16 binades within a row, opposed to the activations)
+ * need TENSOR_F8 or FMA. */
 
 /* Same contract as mxfp4_moe_ffn with an explicit kernel variant. */
 int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,

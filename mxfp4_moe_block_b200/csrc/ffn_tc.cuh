@@ -87,15 +87,15 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   const uint64_t limit = *(volatile unsigned long long *)&g_wait_limit_ns;
-  for (uint32_t i = 0;; ++i) {
+  // each try_wait may itself suspend the thread for a while, so the flag
+  // and the clock are checked after every one of them
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63) {
-      if (*abort) return false;
-      if (global_ns() - t0 >= limit) {
-        raise_status(MOE_DEV_TIMEOUT);
-        *abort = 1;
-        return false;
-      }
+    if (*abort) return false;
+    if (global_ns() - t0 >= limit) {
+      raise_status(MOE_DEV_TIMEOUT);
+      *abort = 1;
+      return false;
     }
   }
 }
@@ -103,9 +103,9 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
 // Wait for the completion of work already issued (abort flag ignored).
 __device__ __noinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
-  for (uint32_t i = 0;; ++i) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && global_ns() - t0 >= kDrainLimitNs) {
+    if (global_ns() - t0 >= kDrainLimitNs) {
       raise_status(MOE_DEV_TIMEOUT);
       return false;
     }
@@ -315,12 +315,19 @@ __device__ __forceinline__ uint32_t to_e2m1(float v) {
   return (uint32_t)__nv_cvt_float_to_fp4(v, __NV_E2M1, cudaRoundNearest) & 0xfu;
 }
 
+// Largest |v| over the warp: non-negative floats order like their bit
+// patterns, so one integer max reduction (redux.sync) replaces a chain of
+// five shuffles.
+__device__ __forceinline__ float warp_absmax(float v) {
+  return __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(fabsf(v))));
+}
+
 // Two E4M3 terms: codes q[0..1] of this lane, scale bytes sb[0..1] (warp-uniform).
 __device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t (&sb)[2]) {
   float r = v;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const float amax = warp_max(fabsf(r));
+    const float amax = warp_absmax(r);
     int s = 0;
     uint32_t c = 0;
     if (amax > 0.f) {
@@ -532,7 +539,7 @@ inline cudaError_t launch_encode_f4(const uint16_t *src, const int32_t *sp, int 
 
 struct TcMaps {
   CUtensorMap a;        // weights [E*rows, K]: box 128 (padded E2M1) or 128 B (packed) x 64 rows
-  CUtensorMap b[5];     // activation terms [T*P, row bytes]: box 128 B x {16,...,256} rows
+  CUtensorMap b[4];     // activation terms [T*P, row bytes]: box 128 B x {16, 32, 64, 128} rows
 };
 
 struct TcArgs {
@@ -543,7 +550,7 @@ struct TcArgs {
   int E, K, rows_per_expert, P;
   int I;                     // GEMM-1: the gate/up split
   int H;                     // y row length (GEMM-2)
-  int b_box[5];              // rows of each B box (clamped to T*P)
+  int b_box[4];              // rows of each B box (clamped to T*P)
   // GEMM-1 outputs
   uint16_t *h;               // [P, I] bf16
   uint8_t *hq;               // activation terms of h
@@ -573,13 +580,16 @@ struct TcCfg {
   static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
   static constexpr int kSfCols =                                    // TMEM columns per stage
       4 * Kd::kKGroups * (Kd::kRowScaledB ? 1 : 1 + kRowChunks);
-  static constexpr int kAcc = BN <= 128 ? 2 : 1;                   // accumulator buffers
   // Independent accumulation chains per buffer: with few B columns each MMA
   // is tiny and a single chain would run at MMA latency; MMA kk of a stage
   // accumulates into chain kk % kChains and the epilogue adds the chains.
   static constexpr int kChains = BN <= 32 ? 4 : BN <= 64 ? 2 : 1;
-  static constexpr int kAccCols = kAcc * kChains * BN;
   static constexpr int kSfbConstCols = Kd::kRowScaledB ? 4 * kRowChunks : 0;
+  // Two accumulator buffers (the epilogue drains one while the MMAs fill the
+  // other) wherever tensor memory holds them beside the scale columns.
+  static constexpr int kAcc =
+      2 * kChains * BN + kStages * kSfCols + kSfbConstCols <= 512 ? 2 : 1;
+  static constexpr int kAccCols = kAcc * kChains * BN;
   static constexpr int kUsed = kAccCols + kStages * kSfCols + kSfbConstCols;
   static constexpr int kTmemCols = kUsed <= 128 ? 128 : kUsed <= 256 ? 256 : 512;
   static_assert(kUsed <= 512, "TMEM budget");
@@ -751,12 +761,21 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
+      // B rows of a tile: one box of 16, 32, 64 or 128 rows, or -- wider
+      // tiles -- a 128-row box and a second one for the rest, so a stage
+      // loads at most 15 rows more than the tile's N.  bsel = box class
+      // (0..3) | (class of the second box + 1) << 3.
+      auto box_class = [](int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; };
       auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel) {
         int e, mt, nB;
         decode(t, e, mt, rowB, nB);
         const int ncol = (nB + 15) & ~15;
-        bsel = ncol <= 16 ? 0 : ncol <= 32 ? 1 : ncol <= 64 ? 2 : ncol <= 128 ? 3 : 4;
+        bsel = ncol <= 128 ? box_class(ncol) : 3 | ((box_class(ncol - 128) + 1) << 3);
         arow = e * a.rows_per_expert + (MODE == 1 ? mt * 64 : mt * 128);
+      };
+      auto b_bytes = [&](int bsel) {
+        const int tail = bsel >> 3;
+        return (uint32_t)(a.b_box[bsel & 7] + (tail ? a.b_box[tail - 1] : 0)) * 128u;
       };
       // the box's inner coordinate is in elements (padded E2M1) or bytes
       // (packed E2M1); both are kt * 128.  Rows 0-63 of the tile, then rows
@@ -768,7 +787,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
                     pol_w);
       };
       auto load_b = [&](int st, int bsel, int rowB, int kt) {
-        tma_load_2d(smem + C::kOffB + st * C::kB, &maps.b[bsel], kt * 128, rowB, &full[st], pol_x);
+        uint8_t *sb = smem + C::kOffB + st * C::kB;
+        tma_load_2d(sb, &maps.b[bsel & 7], kt * 128, rowB, &full[st], pol_x);
+        if (bsel >> 3)
+          tma_load_2d(sb + 128 * 128, &maps.b[(bsel >> 3) - 1], kt * 128, rowB + 128, &full[st],
+                      pol_x);
       };
       // Tile sequence: blockIdx.x first, then gridDim.x + (the counter's next
       // value) -- a CTA whose tiles went fast takes more.  Each index is
@@ -793,7 +816,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         tile_geom(blockIdx.x, arow, rowB, bsel);
         npre = min(C::kStages, ksteps);
         for (int kt = 0; kt < npre; ++kt) {
-          mbar_expect_tx(&full[kt], Kd::kABytes + (uint32_t)a.b_box[bsel] * 128u);
+          mbar_expect_tx(&full[kt], Kd::kABytes + b_bytes(bsel));
           load_a(kt, arow, kt);
         }
         pdl_wait();
@@ -812,7 +835,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         if (!publish(t_next < n_tiles ? t_next : n_tiles)) break;
         int arow, rowB, bsel;
         tile_geom(t, arow, rowB, bsel);
-        const uint32_t bbytes = (uint32_t)a.b_box[bsel] * 128u;
+        const uint32_t bbytes = b_bytes(bsel);
         for (int kt = t == (int)blockIdx.x ? npre : 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
@@ -1353,19 +1376,20 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a.hq = hq;
   a.hs = hs;
   a.y = f.y;
-  for (int i = 0; i < 5; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
+  // B boxes of 16, 32, 64 and 128 rows (wider tiles load two)
+  for (int i = 0; i < 4; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
 
   // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]; GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   TcMaps maps1, maps2;
   const TcMapKey key{KIND, BN, dev, H, I, E, P, f.w13c, f.w2c, xq, hq};
   if (!tc_map_cache().find(key, maps1, maps2)) {
     if (!make_weight_map<KIND>(&maps1.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 4; ++i)
       if (!make_map(&maps1.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
                     a.b_box[i]))
         return MOE_ERR_CUDA;
     if (!make_weight_map<KIND>(&maps2.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 4; ++i)
       if (!make_map(&maps2.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
                     a.b_box[i]))
         return MOE_ERR_CUDA;
@@ -1423,6 +1447,7 @@ inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   if (want <= 32) return tc_run<KIND, 32>(f, ws, sms, s);
   if (want <= 64) return tc_run<KIND, 64>(f, ws, sms, s);
   if (want <= 128) return tc_run<KIND, 128>(f, ws, sms, s);
+  if (want <= 192) return tc_run<KIND, 192>(f, ws, sms, s);
   return tc_run<KIND, 256>(f, ws, sms, s);
 }
 

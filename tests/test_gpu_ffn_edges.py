@@ -1,0 +1,187 @@
+"""GPU FFN parity at the edges of the MXFP4 format and of the activation
+encodings, against the oracle, for every kernel variant.
+
+The seeded workloads draw scale bytes in [120, 130] and N(0,1) activations;
+these cases do not.  Each compares every output row (h and y) with the
+oracle at the FFN tolerance (rel-L2 <= 2e-3, max-abs <= 1e-2 max|ref|):
+
+A  format edge values: E8M0 scale bytes 0 (the subnormal 2^-127), 1, 126,
+   127, 128 beside ordinary ones, whole 32-element blocks of +0, -0, +6 and
+   -6 codes, and experts that no token selects interleaved with busy ones;
+   an expert intermediate of 384 (a multiple of 128, not of 256), where the
+   automatic choice must take kind::mxf8f6f4.
+B  activation rows whose 32-element blocks span 2^-12 .. 2^12 (a range of
+   2^24 and more inside one row) against ordinary weights.
+C  the same with weight scales inversely matched to the activation blocks
+   (every block contributes alike) over a 2^16 range: the domain the
+   kind::mxf4 encoding (eight terms, one scale per row and term) covers.
+D  scale-matched blocks over the whole E8M0 range (bytes 0 .. 254): the
+   per-32-element-block encodings (FMA dequantisation, kind::mxf8f6f4) only;
+   kind::mxf4 represents each row to ~2^-16 of its largest element and is
+   documented as outside its domain there.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_moe_block_b200 as mm
+from mxfp4_moe_block_b200 import synth
+from oracle import moe as omoe
+
+from gpu_helpers import assert_ffn_close, bf16_to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ALL = [mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_AUTO]
+NAMES = {mm.FFN_FMA: "fma", mm.FFN_TENSOR_F8: "mxf8f6f4", mm.FFN_TENSOR_F4: "mxf4",
+         mm.FFN_AUTO: "auto"}
+
+
+@pytest.fixture(autouse=True)
+def clean_status():
+    mm.moe_clear_device_status()
+    yield
+
+
+class EdgeLayer:
+    """One layer's weights and inputs, drawn by the seeded generator and then
+    edited in numpy (the same arrays go to the device and to the oracle)."""
+
+    def __init__(self, sh, empty=()):
+        E = sh.E
+        self.sh = sh
+        self.w13c = np.stack([synth.weight_codes_np(sh, "w13", e) for e in range(E)])
+        self.w13s = np.stack([synth.weight_scales_np(sh, "w13", e) for e in range(E)])
+        self.w2c = np.stack([synth.weight_codes_np(sh, "w2", e) for e in range(E)])
+        self.w2s = np.stack([synth.weight_scales_np(sh, "w2", e) for e in range(E)])
+        self.x = synth.bf16_bits_to_f32(synth.x_bf16_bits(sh)).astype(np.float64)
+        self.logits = synth.router_logits(sh)
+        self.logits[:, list(empty)] = -1e4          # never selected
+        self.rng = np.random.default_rng(sh.seed)
+
+    def oracle_weights(self, e):
+        return self.w13c[e], self.w13s[e], self.w2c[e], self.w2s[e]
+
+    def run(self, variant):
+        sh = self.sh
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+        xb = synth.f32_to_bf16_bits(self.x.astype(np.float32))
+        assert np.array_equal(synth.bf16_bits_to_f32(xb), self.x.astype(np.float32)), \
+            "activations must be bf16 values"
+        x = t(xb.view(np.int16)).view(torch.bfloat16)
+        w = [t(a) for a in (self.w13c, self.w13s, self.w2c, self.w2s)]
+        idx, tw = mm.moe_route_topk(t(self.logits), sh.k)
+        off, sp, pr = mm.moe_permute(idx, sh.E)
+        y, ws = mm.mxfp4_moe_ffn(x, sh.k, *w, off, sp, variant=variant)
+        torch.cuda.synchronize()
+        h = bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I))
+        return off.cpu().numpy(), sp.cpu().numpy(), h, y.cpu().numpy().astype(np.float64)
+
+    def check(self, variants, what):
+        sh = self.sh
+        ridx, _, _ = omoe.route_topk(self.logits, sh.k)
+        roff, rsp, _ = omoe.permute(ridx, sh.E)
+        h_ref, y_ref = omoe.moe_ffn(self.x, sh.k, sh.I, self.oracle_weights, roff, rsp)
+        assert np.all(np.isfinite(y_ref))
+        for v in variants:
+            off, sp, h, y = self.run(v)
+            assert np.array_equal(off, roff) and np.array_equal(sp, rsp)
+            r = assert_ffn_close(y, y_ref, f"{what} {NAMES[v]} y")
+            assert_ffn_close(h, h_ref, f"{what} {NAMES[v]} h")
+            print(f"[{what}] {NAMES[v]}: y rel-L2 {r[0]:.2e}")
+            assert mm.moe_get_device_status() == (0, 0)
+
+
+def _edge_values(L):
+    """Scale bytes 0, 1, 126, 127, 128 scattered over ordinary ones; whole
+    blocks of +0 / -0 / +6 / -6 codes."""
+    rng = L.rng
+    for s in (L.w13s, L.w2s):
+        pick = rng.random(s.shape)
+        s[pick < 0.04] = 0
+        s[(pick >= 0.04) & (pick < 0.08)] = 1
+        mid = (pick >= 0.08) & (pick < 0.3)
+        s[mid] = rng.choice(np.array([126, 127, 128], np.uint8), size=int(mid.sum()))
+    for c in (L.w13c, L.w2c):
+        E, R, KB = c.shape                      # KB = K/2 bytes; a block = 16 bytes
+        blocks = c.reshape(E, R, KB // 16, 16)
+        pick = rng.random(blocks.shape[:3])
+        blocks[pick < 0.05] = 0x00               # +0 +0
+        blocks[(pick >= 0.05) & (pick < 0.1)] = 0x88   # -0 -0
+        blocks[(pick >= 0.1) & (pick < 0.15)] = 0x77   # +6 +6
+        blocks[(pick >= 0.15) & (pick < 0.2)] = 0xFF   # -6 -6
+
+
+def test_format_edge_values_auto_takes_mxf8f6f4():
+    """I = 384: kind::mxf4 is unavailable (needs multiples of 256), the
+    automatic choice takes kind::mxf8f6f4."""
+    sh = synth.Shape("edges", H=1024, I=384, E=16, k=4, S=2, K=8, V=64, seed=2101)
+    L = EdgeLayer(sh, empty=(1, 4, 9, 14))
+    _edge_values(L)
+    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_AUTO], "edges I=384")
+    with pytest.raises(mm.MoeError) as ei:
+        L.run(mm.FFN_TENSOR_F4)
+    assert ei.value.status == 2
+
+
+def test_format_edge_values_every_variant():
+    sh = synth.Shape("edges2", H=1024, I=512, E=16, k=4, S=2, K=8, V=64, seed=2102)
+    L = EdgeLayer(sh, empty=(0, 3, 7, 15))
+    _edge_values(L)
+    L.check(ALL, "edges I=512")
+
+
+def _block_magnitudes(L, exps):
+    """Scale each 32-element block b of every activation row by 2^exps[b]
+    (rounded to bf16 afterwards)."""
+    from oracle import mxfp4 as omx
+    L.x = omx.round_bf16(L.x * np.repeat(np.exp2(exps.astype(np.float64)), 32)[None, :])
+
+
+def test_activation_rows_spanning_2_24_and_more():
+    sh = synth.Shape("xrange", H=2048, I=512, E=8, k=2, S=2, K=8, V=64, seed=2103)
+    L = EdgeLayer(sh)
+    exps = L.rng.integers(-12, 13, sh.H // 32)
+    exps[0], exps[1] = -12, 12                    # the row spans at least 2^24
+    _block_magnitudes(L, exps)
+    L.check(ALL, "x range 2^24")
+
+
+def _matched_scales(L, exps):
+    """W13's 32-column block b gets scale byte 127 - exps[b] in every row, so
+    that each block's products come out alike (an activation channel that is
+    large meets small weights); W2 keeps ordinary scales."""
+    sb = (127 - exps).astype(np.int64)
+    assert sb.min() >= 0 and sb.max() <= 254
+    L.w13s[:] = sb.astype(np.uint8)[None, None, :]
+
+
+def test_scale_matched_blocks_within_the_mxf4_domain():
+    sh = synth.Shape("matched16", H=2048, I=512, E=8, k=2, S=2, K=8, V=64, seed=2104)
+    L = EdgeLayer(sh)
+    exps = L.rng.integers(-8, 9, sh.H // 32)      # a 2^16 range
+    exps[0], exps[1] = -8, 8
+    _block_magnitudes(L, exps)
+    _matched_scales(L, exps)
+    L.check(ALL, "matched 2^16")
+
+
+def test_scale_matched_blocks_over_the_whole_e8m0_range():
+    """Scale bytes 0, 1, ... 254 (the E8M0 subnormal 2^-127 included) met by
+    activations 2^127 ... 2^-127: only per-block-scaled encodings represent
+    such rows.  Codes of the 2^127 blocks stay within +-1.5 so that every
+    weight is a finite bf16 value."""
+    sh = synth.Shape("matchedall", H=2048, I=512, E=8, k=2, S=2, K=8, V=64, seed=2105)
+    L = EdgeLayer(sh)
+    sb = np.array([0, 1, 60, 127, 200, 254], np.int64)[L.rng.integers(0, 6, sh.H // 32)]
+    sb[:6] = [0, 1, 60, 127, 200, 254]
+    exps = 127 - sb
+    # keep activations finite in bf16 at 2^127: |N(0,1)| clipped to 1.9
+    L.x = np.clip(L.x, -1.9, 1.9)
+    _block_magnitudes(L, exps)
+    L.w13s[:] = sb.astype(np.uint8)[None, None, :]
+    big = np.repeat(sb == 254, 16)                # byte columns of the 2^127 blocks
+    c = L.w13c[:, :, big]
+    lo, hi = c & 0x0F, c >> 4
+    L.w13c[:, :, big] = ((lo & 0x0B) | ((hi & 0x0B) << 4)).astype(np.uint8)   # |value| <= 1.5
+    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8], "matched full E8M0")

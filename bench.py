@@ -59,7 +59,8 @@ def parse(argv=None):
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--per-config", default=",".join(PER_CONFIG),
-                    help="comma-separated workloads for the per_config object")
+                    help="comma-separated workloads for the per_config object (the "
+                         "quantiser is always measured; 'none' for it alone)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override the expert count (smaller cases for profiler captures)")
     return ap.parse_args(argv)
@@ -813,7 +814,8 @@ def main():
     if world == 1:
         if not args.no_per_config:
             pc = {}
-            for name in [n for n in args.per_config.split(",") if n and n != sh.name]:
+            for name in [n for n in args.per_config.split(",")
+                         if n in synth.SHAPES and n != sh.name]:
                 pc[name] = measure_config(name, variant, min(args.steps, 20), args.warmup, dev,
                                           peaks, clocks, not args.no_cpu_baseline)
             pc["quantize"] = measure_quantize(dev, peaks)

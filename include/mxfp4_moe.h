@@ -168,9 +168,17 @@ enum {
                             TENSOR_F8                                             */
   MOE_FFN_TENSOR_F8 = 3, /* kind::mxf8f6f4: padded E2M1 weights x two E4M3
                             activation terms with E8M0 block scales               */
-  MOE_FFN_TENSOR_F4 = 4  /* kind::mxf4: packed E2M1 weights x eight E2M1
+  MOE_FFN_TENSOR_F4 = 4, /* kind::mxf4: packed E2M1 weights x eight E2M1
                             activation terms with one scale per row and term
                             (H, I multiples of 256, at most 8192)                 */
+  MOE_FFN_TENSOR_FUSED = 5 /* TENSOR_F4 with both GEMMs in one persistent
+                            launch (I <= 4096): the last GEMM-1 tile of each
+                            expert's token block encodes its h rows and
+                            publishes them by a flag, and GEMM-2 tiles wait
+                            for that flag (bounded) instead of for the end
+                            of a launch -- the first piece of a persistent
+                            verify kernel, after the persistent engine of
+                            [P4] (prior art).  Same results as TENSOR_F4.   */
 };
 /* Accuracy domain of the activation encodings.  FMA and TENSOR_F8 represent
  * every 32-element block of an activation row on its own scale, so they meet

@@ -9,9 +9,9 @@
 // (16 bytes = 32 E2M1 codes = exactly one MX block with one scale byte), so
 // each warp-wide load moves 512 contiguous bytes of a row.  Per chunk the
 // lane decodes two codes at a time (hardware E2M1x2 -> f16x2 conversion, then
-// to float), accumulates even/odd products with packed f32x2 FMAs, scales the
-// block's partial sum by its E8M0 scale (an exact power of two) and adds it
-// to the row total; the warp reduces at the end.  Activations are read as
+// to float), multiplies the pair by the block's E8M0 scale (an exact power of
+// two: the dequantised weights) and accumulates even/odd products with packed
+// f32x2 FMAs; the warp reduces at the end.  Activations are read as
 // float (converted once by x_to_f32_kernel; GEMM-1 stores h in float too).
 // Items (expert, row group) are dealt to warps in contiguous runs, so a
 // warp's consecutive items share the expert and its activations stay in L1.
@@ -117,19 +117,24 @@ __device__ __forceinline__ void fma_rows(const uint8_t *__restrict__ wc,
     }
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
+      // each code pair times the block's scale (exact: a power of two) is
+      // the dequantised weight pair, so every product is weight x activation
+      // -- no block partial sum outside the range of the result
       float2 part[NT];
 #pragma unroll
       for (int j = 0; j < NT; ++j) part[j] = make_float2(0.f, 0.f);
       const uint32_t qw[4] = {q[r].x, q[r].y, q[r].z, q[r].w};
 #pragma unroll
       for (int b = 0; b < 16; ++b) {
-        const float2 wv = e2m1x2_to_f32x2(qw[b >> 2] >> (8 * (b & 3)));
+        const float s = e8m0_to_f32(sc[r]);
+        float2 wv = e2m1x2_to_f32x2(qw[b >> 2] >> (8 * (b & 3)));
+        wv.x *= s;
+        wv.y *= s;
 #pragma unroll
         for (int j = 0; j < NT; ++j) part[j] = ffma2(wv, xv[j][b], part[j]);
       }
-      const float s = e8m0_to_f32(sc[r]);
 #pragma unroll
-      for (int j = 0; j < NT; ++j) acc[r][j] = fmaf(part[j].x + part[j].y, s, acc[r][j]);
+      for (int j = 0; j < NT; ++j) acc[r][j] += part[j].x + part[j].y;
     }
   }
 #pragma unroll

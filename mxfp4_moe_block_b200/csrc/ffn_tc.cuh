@@ -112,6 +112,50 @@ __device__ __noinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
   }
 }
 
+// Flags in global memory between the CTAs of one launch (the fused FFN):
+// release / acquire at GPU scope, and a bounded wait like the barrier waits.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// atomic add with acquire-release semantics at GPU scope; returns the old value
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int *p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ float ld_weak_f32(const float *p) {
+  float v;
+  asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Generic-proxy writes before, async-proxy (TMA) reads after -- or the other
+// way round -- of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __noinline__ bool wait_flag(const int *f, volatile int *abort) {
+  if (ld_acquire_gpu(f)) return true;
+  const uint64_t t0 = global_ns();
+  const uint64_t limit = *(volatile unsigned long long *)&g_wait_limit_ns;
+  for (;;) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(f)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 >= limit) {
+      raise_status(MOE_DEV_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Inline first try; the bounded slow path only when the phase is not done.
 __device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity,
                                                volatile int *abort) {
@@ -340,8 +384,9 @@ __device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t
   }
 }
 
-// Kind of tensor-core MMA used by the FFN.
-enum TcKind { KIND_F8 = 0, KIND_F4 = 1 };
+// Kind of tensor-core MMA used by the FFN (KIND_F4_FUSED: kind::mxf4, both
+// GEMMs in one launch -- a host-side choice only; the kernels see KIND_F4).
+enum TcKind { KIND_F8 = 0, KIND_F4 = 1, KIND_F4_FUSED = 2 };
 constexpr int kF4Terms = 8;     // E2M1 terms per activation row (kind::mxf4)
 
 template <int KIND>
@@ -408,16 +453,18 @@ template <int NT>
 __global__ void __launch_bounds__(ENC_THREADS)
 encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp, int k,
                       int K, uint8_t *__restrict__ q, float *__restrict__ rs, int early_trigger,
-                      int *counters) {
+                      int *counters, int ncounters) {
   // early_trigger: the next kernel (GEMM-2) may start streaming its weights
   // while this one still waits for GEMM-1; it reads our output only after
   // its own wait, and nothing of GEMM-1's before it
   if (early_trigger) pdl_trigger();
   pdl_wait();
   if (!early_trigger) pdl_trigger();
-  // the GEMMs' tile counters for this call (GEMM-1 reads its own only after
-  // this kernel completed; GEMM-2 after the next one did)
-  if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
+  // the GEMMs' tile counters for this call, and the fused FFN's B-tile
+  // counters and flags (GEMM-1 reads its own only after this kernel
+  // completed; GEMM-2 after the next one did)
+  if (counters && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const uint16_t *row = src + (size_t)(sp ? __ldg(sp + r) / k : r) * K;
@@ -468,11 +515,12 @@ template <int NT, int PPL>
 __global__ void __launch_bounds__(128)
 encode_rows_f4_warp_kernel(const uint16_t *__restrict__ src, const int32_t *__restrict__ sp,
                            int k, int P, uint8_t *__restrict__ q, float *__restrict__ rs,
-                           int early_trigger, int *counters) {
+                           int early_trigger, int *counters, int ncounters) {
   if (early_trigger) pdl_trigger();
   pdl_wait();
   if (!early_trigger) pdl_trigger();
-  if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
+  if (counters && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
   constexpr int K = 64 * PPL;
   const int lane = threadIdx.x & 31;
   const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -507,6 +555,51 @@ encode_rows_f4_warp_kernel(const uint16_t *__restrict__ src, const int32_t *__re
   }
 }
 
+// The same encoding of one bf16 row of K <= 4096 elements by the 128 threads
+// of one epilogue warp group (the fused FFN's last GEMM-1 tile of a B tile
+// encodes that tile's h rows).  The row is read through L2 (ld.global.cg):
+// other CTAs of the same launch wrote parts of it.  red: 8 floats of shared
+// memory (two sets of four, alternating by term).
+constexpr int GRP_ENC_MAX_PAIRS = 16;
+template <int NT>
+__device__ __forceinline__ void encode_row_f4_group(const uint16_t *row, int K, uint8_t *q,
+                                                    float *rs, int grp, float *red) {
+  const int tid = (threadIdx.x & 127), lane = tid & 31, w = tid >> 5;
+  const int npairs = K / 2;
+  float v[2 * GRP_ENC_MAX_PAIRS];
+#pragma unroll
+  for (int j = 0; j < GRP_ENC_MAX_PAIRS; ++j) {
+    const int i = tid + 128 * j;
+    const uint32_t pr = i < npairs ? __ldcg(reinterpret_cast<const unsigned int *>(row) + i) : 0u;
+    v[2 * j] = bf16_lo(pr);
+    v[2 * j + 1] = bf16_hi(pr);
+  }
+#pragma unroll 1
+  for (int t = 0; t < NT; ++t) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2 * GRP_ENC_MAX_PAIRS; ++j) m = fmaxf(m, fabsf(v[j]));
+    m = warp_absmax(m);
+    if (lane == 0) red[(t & 1) * 4 + w] = m;
+    group_sync(grp);
+    const float *rr = red + (t & 1) * 4;
+    const float amax = fmaxf(fmaxf(rr[0], rr[1]), fmaxf(rr[2], rr[3]));
+    const int sexp = amax > 0.f ? e2m1_block_exp(amax) : 0;
+    const float inv = pow2f(-sexp), sc = pow2f(sexp);
+    uint8_t *qrow = q + (size_t)t * (K / 2);
+#pragma unroll
+    for (int j = 0; j < GRP_ENC_MAX_PAIRS; ++j) {
+      const int i = tid + 128 * j;
+      const uint32_t c0 = to_e2m1(v[2 * j] * inv), c1 = to_e2m1(v[2 * j + 1] * inv);
+      const float2 d = e2m1x2_to_f32x2(c0 | (c1 << 4));
+      v[2 * j] -= d.x * sc;
+      v[2 * j + 1] -= d.y * sc;
+      if (i < npairs) qrow[i] = (uint8_t)(c0 | (c1 << 4));
+    }
+    if (tid == 0) rs[t] = sc;
+  }
+}
+
 // Launch a row encoder: a CTA per row (shortest latency: a row's work
 // spread over 256 threads) for a few rows, a warp per row (no barriers, the
 // most rows per SM) once there are hundreds.
@@ -514,24 +607,24 @@ constexpr size_t ENC_WARP_MIN_ROWS = 512;
 template <int NT>
 inline cudaError_t launch_encode_f4(const uint16_t *src, const int32_t *sp, int k, int K,
                                    size_t P, uint8_t *q, float *rs, int early_trigger,
-                                   int *counters, cudaStream_t s) {
+                                   int *counters, int ncounters, cudaStream_t s) {
   const unsigned g4 = (unsigned)((P + 3) / 4);
   switch (P >= ENC_WARP_MIN_ROWS ? K : 0) {
     case 256:
       return launch_pdl(encode_rows_f4_warp_kernel<NT, 4>, g4, 128, 0, s, src, sp, k, (int)P, q,
-                        rs, early_trigger, counters);
+                        rs, early_trigger, counters, ncounters);
     case 512:
       return launch_pdl(encode_rows_f4_warp_kernel<NT, 8>, g4, 128, 0, s, src, sp, k, (int)P, q,
-                        rs, early_trigger, counters);
+                        rs, early_trigger, counters, ncounters);
     case 1024:
       return launch_pdl(encode_rows_f4_warp_kernel<NT, 16>, g4, 128, 0, s, src, sp, k, (int)P, q,
-                        rs, early_trigger, counters);
+                        rs, early_trigger, counters, ncounters);
     case 2048:
       return launch_pdl(encode_rows_f4_warp_kernel<NT, 32>, g4, 128, 0, s, src, sp, k, (int)P, q,
-                        rs, early_trigger, counters);
+                        rs, early_trigger, counters, ncounters);
     default:
       return launch_pdl(encode_rows_f4_kernel<NT>, (unsigned)P, ENC_THREADS, 0, s, src, sp, k, K,
-                        q, rs, early_trigger, counters);
+                        q, rs, early_trigger, counters, ncounters);
   }
 }
 
@@ -560,6 +653,10 @@ struct TcArgs {
   // tiles past the first wave are handed out by this counter (zeroed by the
   // encode kernel that runs first in the call)
   int *tile_counter;
+  // fused FFN: per B tile, GEMM-1 tiles finished and the GEMM-2 operand's
+  // readiness flag (zeroed by the same encode kernel)
+  int *bt_done;
+  int *bt_ready;
 };
 
 constexpr int kMaxStages = 12;
@@ -629,9 +726,19 @@ __device__ __forceinline__ int ring_read(uint64_t *ring_full, uint64_t *ring_emp
   return t;
 }
 
+// MODE 1: GEMM-1 + SwiGLU (maps, a); MODE 2: GEMM-2 (maps, a); MODE 3: the
+// fused FFN, one launch over every GEMM-1 tile (maps, a) and then every
+// GEMM-2 tile (maps2, a2) -- phase 0 and phase 1 of the tile sequence.  The
+// last GEMM-1 tile of a B tile (the rows of one expert in one B-tile slot)
+// encodes those h rows into the GEMM-2 operand and raises the B tile's
+// readiness flag; a GEMM-2 tile's producer waits for the flag (bounded)
+// before loading its B operand.  Every CTA is resident at once (one per SM)
+// and tiles are taken in increasing order, so every GEMM-1 tile a waiting
+// GEMM-2 tile needs is held by a running CTA.
 template <int KIND, int MODE, int BN>
 __global__ void __launch_bounds__(TcKindCfg<KIND>::kThreads, 1)
-tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
+tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcArgs a,
+               const __grid_constant__ TcMaps maps2, const __grid_constant__ TcArgs a2) {
   using C = TcCfg<KIND, BN>;
   using Kd = TcKindCfg<KIND>;
   constexpr int T = Kd::kTerms;
@@ -661,9 +768,17 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   int *s_pre = reinterpret_cast<int *>(smem + C::kOffTab + 1026 * 2);   // tile prefix
   int *s_r0 = s_pre + 1025;        // first sorted row of each active expert (+ total)
 
+  // the fused FFN's encode scratch: the last-tile flag and the row maxima
+  volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::kOffBar + 512);
+  float *s_red = reinterpret_cast<float *>(smem + C::kOffBar + 512 + 16);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mtiles = MODE == 1 ? a.I / 64 : a.rows_per_expert / 128;
-  const int ksteps = a.K / Kd::kStageK;
+  // m-blocks of a B tile and K stages, per phase (phase 1: MODE 3 only)
+  const int mt1 = MODE == 2 ? a.rows_per_expert / 128 : a.I / 64;
+  const int mt2 = a2.rows_per_expert / 128;
+  const int ks1 = a.K / Kd::kStageK, ks2 = a2.K / Kd::kStageK;
+  // the table's prefix is in tiles (MODES 1, 2) or in B tiles (MODE 3)
+  const int mtiles = MODE == 3 ? 1 : mt1;
 
   // tile table: active experts and the prefix of their tile counts
   if (warp == 0) {
@@ -730,26 +845,44 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_act = s_act[1024];
-  const int n_tiles = s_pre[n_act];
+  const int n_bt = s_pre[n_act];
+  const int n1 = MODE == 3 ? n_bt * mt1 : n_bt;          // tiles of phase 0
+  const int n_tiles = MODE == 3 ? n1 + n_bt * mt2 : n_bt;
+  auto phase_of = [&](int t) { return (MODE == 3 && t >= n1) ? 1 : 0; };
+  auto mode_of = [&](int ph) { return MODE == 3 ? 1 + ph : MODE; };
+  auto ksteps_of = [&](int ph) { return ph ? ks2 : ks1; };
 
-  // tile index -> (expert, m-block, first B row, B rows in the tile)
-  // Every role walks its tiles in increasing order, so the active-expert
-  // index only moves forward: a linear advance from the last position, all
-  // from shared memory.
-  int dpos = 0;
-  auto decode = [&](int t, int &e, int &mt, int &rowB, int &nB) {
+  // tile index -> (expert, m-block, first B row, B rows in the tile, phase,
+  // global B-tile index).  Every role walks its tiles in increasing order,
+  // so within a phase the active-expert index only moves forward: a linear
+  // advance from the last position, all from shared memory.
+  struct Tile {
+    int e, mt, rowB, nB, ph, g;
+  };
+  int dpos = 0, dph = 0;
+  auto decode = [&](int t) {
+    Tile r;
+    r.ph = phase_of(t);
+    const int tl = r.ph ? t - n1 : t;
+    const int mtl = MODE == 3 ? (r.ph ? mt2 : mt1) : 1;
+    if (r.ph != dph) {
+      dpos = 0;
+      dph = r.ph;
+    }
     int lo = dpos;
-    while (lo + 1 < n_act && s_pre[lo + 1] <= t) ++lo;
+    while (lo + 1 < n_act && s_pre[lo + 1] * mtl <= tl) ++lo;
     dpos = lo;
-    e = s_act[lo];
+    r.e = s_act[lo];
     const int r0 = s_r0[lo];
     const int ne = s_r0[lo + 1] - r0;
     const int nt_cnt = (T * ne + BN - 1) / BN;
-    const int local = t - s_pre[lo];
-    mt = local / nt_cnt;
+    const int local = tl - s_pre[lo] * mtl;
+    r.mt = local / nt_cnt;
     const int nt = local % nt_cnt;
-    rowB = T * r0 + nt * BN;
-    nB = min(BN, T * ne - nt * BN);
+    r.g = s_pre[lo] + nt;
+    r.rowB = T * r0 + nt * BN;
+    r.nB = min(BN, T * ne - nt * BN);
+    return r;
   };
 
   int w_arrived = 0;   // stages an A-scale writer warp has released (abort drain)
@@ -766,12 +899,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       // loads at most 15 rows more than the tile's N.  bsel = box class
       // (0..3) | (class of the second box + 1) << 3.
       auto box_class = [](int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; };
-      auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel) {
-        int e, mt, nB;
-        decode(t, e, mt, rowB, nB);
-        const int ncol = (nB + 15) & ~15;
+      auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel, int &ph, int &g) {
+        const Tile tl = decode(t);
+        const int ncol = (tl.nB + 15) & ~15;
         bsel = ncol <= 128 ? box_class(ncol) : 3 | ((box_class(ncol - 128) + 1) << 3);
-        arow = e * a.rows_per_expert + (MODE == 1 ? mt * 64 : mt * 128);
+        rowB = tl.rowB;
+        ph = tl.ph;
+        g = tl.g;
+        const int rpe = ph ? a2.rows_per_expert : a.rows_per_expert;
+        arow = tl.e * rpe + (mode_of(ph) == 1 ? tl.mt * 64 : tl.mt * 128);
       };
       auto b_bytes = [&](int bsel) {
         const int tail = bsel >> 3;
@@ -780,18 +916,30 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       // the box's inner coordinate is in elements (padded E2M1) or bytes
       // (packed E2M1); both are kt * 128.  Rows 0-63 of the tile, then rows
       // 64-127 (GEMM-1: gate, then up).
-      auto load_a = [&](int st, int arow, int kt) {
+      auto load_a = [&](int st, int arow, int kt, int ph) {
         uint8_t *sa = smem + st * C::kA;
-        tma_load_2d(sa, &maps.a, kt * 128, arow, &full[st], pol_w);
-        tma_load_2d(sa + 64 * 128, &maps.a, kt * 128, arow + (MODE == 1 ? a.I : 64), &full[st],
+        const CUtensorMap *m = ph ? &maps2.a : &maps.a;
+        tma_load_2d(sa, m, kt * 128, arow, &full[st], pol_w);
+        tma_load_2d(sa + 64 * 128, m, kt * 128, arow + (mode_of(ph) == 1 ? a.I : 64), &full[st],
                     pol_w);
       };
-      auto load_b = [&](int st, int bsel, int rowB, int kt) {
+      auto load_b = [&](int st, int bsel, int rowB, int kt, int ph) {
         uint8_t *sb = smem + C::kOffB + st * C::kB;
-        tma_load_2d(sb, &maps.b[bsel & 7], kt * 128, rowB, &full[st], pol_x);
+        const CUtensorMap *mb = ph ? maps2.b : maps.b;
+        tma_load_2d(sb, &mb[bsel & 7], kt * 128, rowB, &full[st], pol_x);
         if (bsel >> 3)
-          tma_load_2d(sb + 128 * 128, &maps.b[(bsel >> 3) - 1], kt * 128, rowB + 128, &full[st],
+          tma_load_2d(sb + 128 * 128, &mb[(bsel >> 3) - 1], kt * 128, rowB + 128, &full[st],
                       pol_x);
+      };
+      // a GEMM-2 tile of the fused FFN: its B operand (h rows encoded by the
+      // last GEMM-1 tile of the same B tile) is published by a flag.  On a
+      // failed wait the loads still go out (the kernel is aborting; what they
+      // read does not matter, and every expect_tx gets its bytes).
+      auto b_ready = [&](int ph, int g) {
+        if (MODE != 3 || !ph) return true;
+        const bool ok = wait_flag(a.bt_ready + g, abort);
+        fence_proxy_async_global();
+        return ok;
       };
       // Tile sequence: blockIdx.x first, then gridDim.x + (the counter's next
       // value) -- a CTA whose tiles went fast takes more.  Each index is
@@ -812,16 +960,17 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       // of A stream in before the wait for the activation operand.
       int npre = 0;
       if ((int)blockIdx.x < n_tiles) {
-        int arow, rowB, bsel;
-        tile_geom(blockIdx.x, arow, rowB, bsel);
-        npre = min(C::kStages, ksteps);
+        int arow, rowB, bsel, ph, g;
+        tile_geom(blockIdx.x, arow, rowB, bsel, ph, g);
+        npre = min(C::kStages, ksteps_of(ph));
         for (int kt = 0; kt < npre; ++kt) {
           mbar_expect_tx(&full[kt], Kd::kABytes + b_bytes(bsel));
-          load_a(kt, arow, kt);
+          load_a(kt, arow, kt, ph);
         }
         pdl_wait();
         pdl_trigger();
-        for (int kt = 0; kt < npre; ++kt) load_b(kt, bsel, rowB, kt);
+        b_ready(ph, g);
+        for (int kt = 0; kt < npre; ++kt) load_b(kt, bsel, rowB, kt, ph);
         issued = npre;
         stage = npre % C::kStages;
         phase = npre == C::kStages ? 1u : 0u;
@@ -833,14 +982,16 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
         // the next tile, published before this one's stages are issued
         const int t_next = (int)gridDim.x + atomicAdd(a.tile_counter, 1);
         if (!publish(t_next < n_tiles ? t_next : n_tiles)) break;
-        int arow, rowB, bsel;
-        tile_geom(t, arow, rowB, bsel);
+        int arow, rowB, bsel, ph, g;
+        tile_geom(t, arow, rowB, bsel, ph, g);
         const uint32_t bbytes = b_bytes(bsel);
+        if (t != (int)blockIdx.x && !b_ready(ph, g)) break;
+        const int ksteps = ksteps_of(ph);
         for (int kt = t == (int)blockIdx.x ? npre : 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
-          load_a(stage, arow, kt);
-          load_b(stage, bsel, rowB, kt);
+          load_a(stage, arow, kt, ph);
+          load_b(stage, bsel, rowB, kt, ph);
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
@@ -854,7 +1005,6 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     // Per stage and 4-scale group g: scale bytes of the 128 A rows (and of
     // the B rows) go straight into the 32 x 16-byte layout of tcgen05.cp:
     // byte 16*(row%32) + 4*(row/32) + (k-block within the group).
-    const uint32_t kb = a.K / 32;            // scale bytes per row
     if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
     // Leave-or-stay decisions are warp-wide, so that every stage this warp
     // signals gets all 32 lanes' arrivals.
@@ -864,18 +1014,22 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     for (int ti = 0; ok; ++ti) {
       const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
       if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
-      int e, mt, rowB, nB;
-      decode(t, e, mt, rowB, nB);
-      const int ebase = e * a.rows_per_expert;
+      const Tile tl = decode(t);
+      const int mt = tl.mt, rowB = tl.rowB, nB = tl.nB;
+      const TcArgs &ap = tl.ph ? a2 : a;       // this phase's operands
+      const uint32_t kb = ap.K / 32;           // scale bytes per row
+      const int ebase = tl.e * ap.rows_per_expert;
       // this lane's four A rows (lane + 32q) for the whole tile
       const uint8_t *src_a[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int i = lane + 32 * q;
-        const int row = MODE == 1 ? ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64)
-                                  : ebase + mt * 128 + i;
-        src_a[q] = a.a_scales + (size_t)row * kb;
+        const int row = mode_of(tl.ph) == 1
+                            ? ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64)
+                            : ebase + mt * 128 + i;
+        src_a[q] = ap.a_scales + (size_t)row * kb;
       }
+      const int ksteps = ksteps_of(tl.ph);
       for (int kt = 0; kt < ksteps; ++kt) {
         if (!__all_sync(FULL, mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
           ok = false;
@@ -894,7 +1048,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             const int i = lane + 32 * q;
             if (!Kd::kRowScaledB && i < nB)
               cp_async4(sfb + 512 * (g * C::kRowChunks + (q >> 2)) + 16 * lane + 4 * (q & 3),
-                        a.b_scales + (size_t)(rowB + i) * kb + koff);
+                        ap.b_scales + (size_t)(rowB + i) * kb + koff);
           }
         }
         cp_async_arrive_noinc(&sfs_full[stage]);
@@ -928,9 +1082,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
       int it = 0;
       for (int t = ring_read(ring_full, ring_empty, ring, it, true, abort, n_tiles);
            t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, true, abort, n_tiles)) {
-        int e, mt, rowB, nB;
-        decode(t, e, mt, rowB, nB);
-        const int ncol = (nB + 15) & ~15;
+        const Tile tl = decode(t);
+        const int ncol = (tl.nB + 15) & ~15;
+        const int ksteps = ksteps_of(tl.ph);
         // the tile's instruction descriptor; MMA kk or-s in its scale byte
         // selector (sf_id, bits 4-5 and 29-30)
         const uint32_t idesc0 =
@@ -1013,6 +1167,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     for (int ti = 0; ok; ++ti) {
       const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
       if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
+      const int ksteps = ksteps_of(phase_of(t));
       for (int kt = 0; kt < ksteps; ++kt) {
         // the MMAs that read this stage's columns last time are done, and the
         // stage's scale bytes are in shared memory
@@ -1054,29 +1209,48 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     for (int it = 0;; ++it) {
       const int t = ring_read(ring_full, ring_empty, ring, it, lane == 0, abort, n_tiles);
       bool ok = t < n_tiles && !*abort;
-      int e = 0, mt = 0, rowB = 0, nB = 0;
-      if (ok) decode(t, e, mt, rowB, nB);
+      Tile tl{0, 0, 0, 0, 0, 0};
+      if (ok) tl = decode(t);
+      const int mt = tl.mt, rowB = tl.rowB, nB = tl.nB;
+      const int md = mode_of(tl.ph);
       const int buf = it % C::kAcc;
       const uint32_t use = (uint32_t)(it / C::kAcc);
       const int ntok = nB / T;                  // tokens in this tile (>= 1 in a tile)
       const int rtok0 = rowB / T;               // sorted row of the tile's first token
-      // the first chunk's row scales do not depend on the accumulator: load
-      // them while the MMAs still run
+      // Row scales of the B terms.  The fused FFN's GEMM-2 tiles read ones
+      // this launch wrote -- after the accumulator wait (which follows the
+      // producer's flag wait) and an acquire of the flag, through L2; all
+      // other tiles load the first chunk's before the wait, while the MMAs
+      // still run.
+      const float *rsb = tl.ph ? a2.b_rowscale : a.b_rowscale;
+      const bool rs_late = MODE == 3 && tl.ph;
+      // scales from an earlier launch: the read-only path; ones this launch
+      // wrote: plain loads after the acquire below (the read-only path may
+      // hold a line another B tile's rows share, read before they were
+      // written)
+      auto ld_rs = [&](const float *p) { return rs_late ? ld_weak_f32(p) : __ldg(p); };
       const int cfirst = 16 * grp;              // this group's first chunk
       float rs0[16];
-      if (Kd::kRowScaledB) {
+      auto load_rs0 = [&]() {
         // (rows past ntok are discarded; with no tile the index stays at 0)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int tok = max(0, min((cfirst + i) / T, ntok - 1));
-          rs0[i] = __ldg(a.b_rowscale + (size_t)(rtok0 + tok) * T + i % T);
+          rs0[i] = ld_rs(rsb + (size_t)(rtok0 + tok) * T + i % T);
         }
-      }
+      };
+      if (Kd::kRowScaledB && !rs_late) load_rs0();
       if (ok) ok = mbar_wait_fast(&acc_full[buf], use & 1, abort);
       // the group's four warps leave together: at the end of the tiles, or
       // when any of them saw the abort flag or a wait run out
       if (!group_all(grp, ok)) break;
       tc_fence_after();
+      if (Kd::kRowScaledB && rs_late) {
+        // one acquire per warp, ordered before the other lanes' reads
+        if (lane == 0) (void)ld_acquire_gpu(a.bt_ready + tl.g);
+        __syncwarp();
+        load_rs0();
+      }
       const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
       if (cfirst >= nB) {
         // no chunk for this group: hand the buffer back at once
@@ -1118,9 +1292,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
               for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], rs0[T * j + u], sum);
             } else {
               const int tok = min(tok0 + j, ntok - 1);     // rows past ntok are discarded
-              const float *rsc = a.b_rowscale + (size_t)(rtok0 + tok) * T;
+              const float *rsc = rsb + (size_t)(rtok0 + tok) * T;
 #pragma unroll
-              for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], __ldg(rsc + u), sum);
+              for (int u = 0; u < T; ++u) sum = fmaf(v[T * j + u], ld_rs(rsc + u), sum);
             }
           } else {
 #pragma unroll
@@ -1128,11 +1302,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
           }
           tok_sum[j] = sum;
         }
-        if (MODE == 2) {
+        if (md == 2) {
           const int m = mt * 128 + 32 * q + lane;
+          float *y = MODE == 3 ? a2.y : a.y;
 #pragma unroll
           for (int j = 0; j < kTokPerLd; ++j)
-            if (tok0 + j < ntok) a.y[(size_t)(rtok0 + tok0 + j) * a.H + m] = tok_sum[j];
+            if (tok0 + j < ntok) y[(size_t)(rtok0 + tok0 + j) * a.H + m] = tok_sum[j];
         } else {
           // Rows 0-63 gate (quarters 0,1), 64-127 up (quarters 2,3).  Quarter
           // q and q+2 hold gate and up of the same 32 rows n; the gate warp
@@ -1163,6 +1338,30 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
             }
           }
           group_sync(grp);
+        }
+      }
+      if (MODE == 3 && md == 1) {
+        // The tile's h columns are written.  Count it; the B tile's last
+        // GEMM-1 tile turns the B tile's h rows (complete now) into the
+        // GEMM-2 operand and publishes them.
+        group_sync(grp);
+        if (q == 0 && lane == 0) {
+          // release: the group's h stores (ordered before by the barrier);
+          // acquire: the other tiles' stores, before this group reads them
+          const int done = atom_add_acq_rel_gpu(a.bt_done + tl.g, 1) + 1;
+          *s_last = done == mt1;
+        }
+        group_sync(grp);
+        if (*s_last) {
+          for (int j = 0; j < ntok; ++j) {
+            const size_t r = (size_t)(rtok0 + j);
+            encode_row_f4_group<T>(a.h + r * a.I, a.I, a.hq + (size_t)T * r * (a.I / 2),
+                                   reinterpret_cast<float *>(a.hs) + (size_t)T * r, grp, s_red);
+          }
+          fence_proxy_async_global();           // TMA loads of another CTA read the rows
+          __threadfence();
+          group_sync(grp);
+          if (q == 0 && lane == 0) st_release_gpu(a.bt_ready + tl.g, 1);
         }
       }
     }
@@ -1212,10 +1411,16 @@ inline size_t tc_scale_bytes(size_t P, int K) {
   const size_t f8 = 2 * P * (size_t)K / 32, f4 = kF4Terms * P * sizeof(float);
   return f8 > f4 ? f8 : f4;
 }
+// Counters of one call: the two GEMMs' tile counters (ints 0, 1), then the
+// fused FFN's per-B-tile done counts and readiness flags.  A B tile holds at
+// least 16 term rows (two tokens) or all of an expert's, so there are at
+// most P/2 + (active experts <= 1024) of them.
+inline size_t tc_bt_max(size_t P) { return P / 2 + 1025; }
+inline size_t tc_counter_ints(size_t P) { return 64 + 2 * tc_bt_max(P); }
 inline size_t tc_workspace_bytes(size_t P, int H, int I) {
   return align256_tc(tc_term_bytes(P, H)) + align256_tc(tc_scale_bytes(P, H)) +
          align256_tc(tc_term_bytes(P, I)) + align256_tc(tc_scale_bytes(P, I)) +
-         256;                                   // the two GEMMs' tile counters
+         align256_tc(tc_counter_ints(P) * sizeof(int));
 }
 
 // The tensor-core variant streams the weights with TMA and needs no
@@ -1277,7 +1482,7 @@ inline bool make_weight_map(CUtensorMap *m, const uint8_t *codes, uint64_t K, ui
 // instantiation, set once per device; a failed set is reported and retried
 // on the next call.  Guarded by a mutex: host threads may make their first
 // call at the same time.
-template <int KIND, int BN>
+template <int KIND, int MODE, int BN>
 inline int tc_attributes(int dev) {
   using C = TcCfg<KIND, BN>;
   static std::mutex mu;
@@ -1285,9 +1490,7 @@ inline int tc_attributes(int dev) {
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(mu);
   if ((done >> dev) & 1ull) return MOE_OK;
-  if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, 1, BN>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess ||
-      cudaFuncSetAttribute(tc_gemm_kernel<KIND, 2, BN>,
+  if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, MODE, BN>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
@@ -1343,8 +1546,12 @@ inline TcMapCache &tc_map_cache() {
   return c;
 }
 
-template <int KIND, int BN>
+// One FFN call on the tensor cores: the x encoder, then GEMM-1 + SwiGLU, the
+// h encoder and GEMM-2 -- or, FUSED (kind::mxf4), the x encoder and one
+// launch of both GEMMs that encodes h itself.
+template <int KIND, int BN, bool FUSED>
 int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
+  static_assert(!FUSED || KIND == KIND_F4, "the fused FFN takes the kind::mxf4 operands");
   using C = TcCfg<KIND, BN>;
   using Kd = TcKindCfg<KIND>;
   constexpr int T = Kd::kTerms;
@@ -1363,42 +1570,60 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  const int st = tc_attributes<KIND, BN>(dev);
+  int st = FUSED ? tc_attributes<KIND, 3, BN>(dev) : tc_attributes<KIND, 1, BN>(dev);
+  if (st == MOE_OK && !FUSED) st = tc_attributes<KIND, 2, BN>(dev);
   if (st != MOE_OK) return st;
 
-  TcArgs a{};
-  a.off = f.off;
-  a.E = E;
-  a.P = (int)P;
-  a.I = I;
-  a.H = H;
-  a.h = f.h;
-  a.hq = hq;
-  a.hs = hs;
-  a.y = f.y;
+  // GEMM-1 (a1): W13 [E*2I, H] x x-terms [T*P, H] -> h; GEMM-2 (a2): W2 [E*H, I]
+  // x h-terms [T*P, I] -> y
+  TcArgs a1{};
+  a1.off = f.off;
+  a1.E = E;
+  a1.P = (int)P;
+  a1.I = I;
+  a1.H = H;
+  a1.h = f.h;
+  a1.hq = hq;
+  a1.hs = hs;
+  a1.y = f.y;
   // B boxes of 16, 32, 64 and 128 rows (wider tiles load two)
-  for (int i = 0; i < 4; ++i) a.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
+  for (int i = 0; i < 4; ++i) a1.b_box[i] = (int)std::min<size_t>(16u << i, T * P);
+  a1.tile_counter = counters;
+  a1.bt_done = counters + 64;
+  a1.bt_ready = counters + 64 + tc_bt_max(P);
+  TcArgs a2 = a1;
+  a1.a_scales = f.w13s;
+  a1.b_scales = xs;
+  a1.b_rowscale = reinterpret_cast<const float *>(xs);
+  a1.K = H;
+  a1.rows_per_expert = 2 * I;
+  a2.a_scales = f.w2s;
+  a2.b_scales = hs;
+  a2.b_rowscale = reinterpret_cast<const float *>(hs);
+  a2.K = I;
+  a2.rows_per_expert = H;
+  a2.tile_counter = counters + 1;
 
-  // GEMM-1: W13 [E*2I, H] x x-terms [T*P, H]; GEMM-2: W2 [E*H, I] x h-terms [T*P, I]
   TcMaps maps1, maps2;
   const TcMapKey key{KIND, BN, dev, H, I, E, P, f.w13c, f.w2c, xq, hq};
   if (!tc_map_cache().find(key, maps1, maps2)) {
     if (!make_weight_map<KIND>(&maps1.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
     for (int i = 0; i < 4; ++i)
       if (!make_map(&maps1.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
-                    a.b_box[i]))
+                    a1.b_box[i]))
         return MOE_ERR_CUDA;
     if (!make_weight_map<KIND>(&maps2.a, f.w2c, I, (uint64_t)E * H)) return MOE_ERR_CUDA;
     for (int i = 0; i < 4; ++i)
       if (!make_map(&maps2.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
-                    a.b_box[i]))
+                    a1.b_box[i]))
         return MOE_ERR_CUDA;
     tc_map_cache().put(key, maps1, maps2);
   }
 
   if (KIND == KIND_F4) {
+    const int ncounters = FUSED ? (int)tc_counter_ints(P) : 2;
     if (launch_encode_f4<T>(f.x, f.sp, f.k, H, P, xq, reinterpret_cast<float *>(xs), 0, counters,
-                            s) != cudaSuccess)
+                            ncounters, s) != cudaSuccess)
       return MOE_ERR_CUDA;
   } else {
     const long blocks = (long)P * (H / 32);
@@ -1408,33 +1633,26 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
   }
 
-  a.a_scales = f.w13s;
-  a.b_scales = xs;
-  a.b_rowscale = reinterpret_cast<const float *>(xs);
-  a.K = H;
-  a.rows_per_expert = 2 * I;
-  a.tile_counter = counters;
-  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a) !=
-      cudaSuccess)
+  if (FUSED) {
+    if (launch_pdl(tc_gemm_kernel<KIND, 3, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a1, maps2,
+                   a2) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a1, maps1,
+                 a1) != cudaSuccess)
     return MOE_ERR_CUDA;
-
   if (KIND == KIND_F4)
     if (launch_encode_f4<T>(f.h, nullptr, 1, I, P, hq, reinterpret_cast<float *>(hs), 1, nullptr,
-                            s) != cudaSuccess)
+                            0, s) != cudaSuccess)
       return MOE_ERR_CUDA;
-  a.a_scales = f.w2s;
-  a.b_scales = hs;
-  a.b_rowscale = reinterpret_cast<const float *>(hs);
-  a.K = I;
-  a.rows_per_expert = H;
-  a.tile_counter = counters + 1;
-  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, Kd::kThreads, C::kSmem, s, maps2, a) !=
-      cudaSuccess)
+  if (launch_pdl(tc_gemm_kernel<KIND, 2, BN>, sms, Kd::kThreads, C::kSmem, s, maps2, a2, maps2,
+                 a2) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
-template <int KIND>
+template <int KIND, bool FUSED>
 inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   const size_t P = (size_t)f.T * f.k;
   const size_t used = P < (size_t)f.E ? P : (size_t)f.E;
@@ -1443,12 +1661,12 @@ inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   // room for the busier experts, and at least 4 tokens per B tile
   size_t want = rows + rows / 2;
   if (want < 4 * terms) want = 4 * terms;
-  if (want <= 16) return tc_run<KIND, 16>(f, ws, sms, s);
-  if (want <= 32) return tc_run<KIND, 32>(f, ws, sms, s);
-  if (want <= 64) return tc_run<KIND, 64>(f, ws, sms, s);
-  if (want <= 128) return tc_run<KIND, 128>(f, ws, sms, s);
-  if (want <= 192) return tc_run<KIND, 192>(f, ws, sms, s);
-  return tc_run<KIND, 256>(f, ws, sms, s);
+  if (want <= 16) return tc_run<KIND, 16, FUSED>(f, ws, sms, s);
+  if (want <= 32) return tc_run<KIND, 32, FUSED>(f, ws, sms, s);
+  if (want <= 64) return tc_run<KIND, 64, FUSED>(f, ws, sms, s);
+  if (want <= 128) return tc_run<KIND, 128, FUSED>(f, ws, sms, s);
+  if (want <= 192) return tc_run<KIND, 192, FUSED>(f, ws, sms, s);
+  return tc_run<KIND, 256, FUSED>(f, ws, sms, s);
 }
 
 // kind::mxf4 (packed FP4 weights, 4 activation terms) when K allows 256-wide
@@ -1468,13 +1686,18 @@ inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int ki
                        f.I <= 2 * ENC_THREADS * ENC_MAX_PAIRS;
     kind = (f4_ok && narrow) ? KIND_F4 : KIND_F8;
   }
-  if (kind == KIND_F4) {
+  if (kind == KIND_F4 || kind == KIND_F4_FUSED) {
     if (f.H % 256 || f.I % 256 || f.H > 2 * ENC_THREADS * ENC_MAX_PAIRS ||
         f.I > 2 * ENC_THREADS * ENC_MAX_PAIRS)
       return MOE_ERR_UNSUPPORTED;
-    return tc_dispatch<KIND_F4>(f, ws, sms, s);
+    if (kind == KIND_F4_FUSED) {
+      // h rows are encoded by one warp group of the fused kernel
+      if (f.I > 2 * 128 * GRP_ENC_MAX_PAIRS) return MOE_ERR_UNSUPPORTED;
+      return tc_dispatch<KIND_F4, true>(f, ws, sms, s);
+    }
+    return tc_dispatch<KIND_F4, false>(f, ws, sms, s);
   }
-  return tc_dispatch<KIND_F8>(f, ws, sms, s);
+  return tc_dispatch<KIND_F8, false>(f, ws, sms, s);
 }
 
 }  // namespace moe

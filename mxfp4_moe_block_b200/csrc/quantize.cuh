@@ -30,48 +30,70 @@ __device__ __forceinline__ uint32_t e2m1_nearest_even(float a) {
          (uint32_t)(a > 5.0f);
 }
 
+// Quantise one group of 8 bf16 (w4 = its 16 bytes) of a 32-element block
+// whose other three groups sit in lanes lane^1, lane^2, lane^3: returns the
+// packed codes, and the block's scale byte in *sb.
+__device__ __forceinline__ uint32_t quantize_group8(const uint4 v, uint32_t *sb) {
+  const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+  // largest magnitude of the block: bf16 bit patterns without the sign
+  // compare like the magnitudes they encode
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m = max(m, max(wd[i] & 0x7fffu, (wd[i] >> 16) & 0x7fffu));
+  m = max(m, __shfl_xor_sync(FULL, m, 1));
+  m = max(m, __shfl_xor_sync(FULL, m, 2));
+  // scale byte = floor(log2 amax) - 2 + 127 = (biased exponent of amax) - 2,
+  // at least 0 (all-zero and tiny blocks); bf16 exponents stop at 254, so
+  // the byte never exceeds 252
+  const int be = (int)(m >> 7);
+  const uint32_t s = (uint32_t)max(0, be - 2);
+  const float inv = __uint_as_float((254u - s) << 23);   // 2^(127 - s), exact
+  uint32_t word = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t b = (i & 1) ? (wd[i >> 1] >> 16) : (wd[i >> 1] & 0xffffu);
+    // |v| * 2^(127 - s) is exact wherever it can reach 0.25 (no overflow:
+    // it stays below 8)
+    const float a = __uint_as_float((b & 0x7fffu) << 16) * inv;
+    const uint32_t c = e2m1_nearest_even(a) | ((b >> 12) & 8u);   // sign -> bit 3
+    word |= c << (4 * i);
+  }
+  *sb = s;
+  return word;
+}
+
 // w: n8 groups of 8 bf16 (n8 = R*K/8); codes: 4 bytes per group; scales: one
-// byte per 4 groups.
+// byte per 4 groups.  Each warp takes QUANT_UNROLL runs of 32 consecutive
+// groups per trip, all loads first, so that each thread keeps QUANT_UNROLL
+// 16-byte loads in flight.
+constexpr int QUANT_UNROLL = 4;
+
 __global__ void __launch_bounds__(QUANT_THREADS)
 mxfp4_quantize_kernel(const uint16_t *__restrict__ w, size_t n8, uint8_t *__restrict__ codes,
                       uint8_t *__restrict__ scales) {
   pdl_wait();
   pdl_trigger();
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
   const unsigned lane = threadIdx.x & 31;
+  const size_t warps = ((size_t)gridDim.x * blockDim.x) >> 5;
+  const size_t wid = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   // the loop bound is warp-uniform (every lane takes part in the shuffles);
   // n8 is a multiple of 4, so the four threads of a block are valid together
-  for (size_t g0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x - lane; g0 < n8; g0 += stride) {
-    const size_t g = g0 + lane;
-    const bool valid = g < n8;
-    const uint4 v = valid ? ld_stream16(w + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-    // largest magnitude of the block: bf16 bit patterns without the sign
-    // compare like the magnitudes they encode
-    uint32_t m = 0;
+  for (size_t r0 = wid * QUANT_UNROLL; r0 * 32 < n8; r0 += warps * QUANT_UNROLL) {
+    uint4 v[QUANT_UNROLL];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) m = max(m, max(wd[i] & 0x7fffu, (wd[i] >> 16) & 0x7fffu));
-    m = max(m, __shfl_xor_sync(FULL, m, 1));
-    m = max(m, __shfl_xor_sync(FULL, m, 2));
-    // scale byte = floor(log2 amax) - 2 + 127 = (biased exponent of amax) - 2,
-    // at least 0 (all-zero and tiny blocks); bf16 exponents stop at 254, so
-    // the byte never exceeds 252
-    const int be = (int)(m >> 7);
-    const uint32_t sb = (uint32_t)max(0, be - 2);
-    const float inv = __uint_as_float((254u - sb) << 23);   // 2^(127 - sb), exact
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t b = (i & 1) ? (wd[i >> 1] >> 16) : (wd[i >> 1] & 0xffffu);
-      // |v| * 2^(127 - sb) is exact wherever it can reach 0.25 (no overflow:
-      // it stays below 8)
-      const float a = __uint_as_float((b & 0x7fffu) << 16) * inv;
-      const uint32_t c = e2m1_nearest_even(a) | ((b >> 12) & 8u);   // sign -> bit 3
-      word |= c << (4 * i);
+    for (int u = 0; u < QUANT_UNROLL; ++u) {
+      const size_t g = (r0 + u) * 32 + lane;
+      v[u] = g < n8 ? ld_stream16(w + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (valid) {
-      *reinterpret_cast<uint32_t *>(codes + 4 * g) = word;
-      if ((g & 3) == 0) scales[g >> 2] = (uint8_t)sb;
+#pragma unroll
+    for (int u = 0; u < QUANT_UNROLL; ++u) {
+      const size_t g = (r0 + u) * 32 + lane;
+      uint32_t sb;
+      const uint32_t word = quantize_group8(v[u], &sb);
+      if (g < n8) {
+        *reinterpret_cast<uint32_t *>(codes + 4 * g) = word;
+        if ((g & 3) == 0) scales[g >> 2] = (uint8_t)sb;
+      }
     }
   }
 }

@@ -40,8 +40,8 @@ def _problem():
     return sh, L, off, sp, h_ref, y_ref
 
 
-@pytest.mark.parametrize("variant", [mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4],
-                         ids=["mxf8f6f4", "mxf4"])
+@pytest.mark.parametrize("variant", [mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED],
+                         ids=["mxf8f6f4", "mxf4", "fused"])
 def test_wait_timeout_reports_and_context_recovers(variant):
     sh, L, off, sp, h_ref, y_ref = _problem()
     timed_out = False

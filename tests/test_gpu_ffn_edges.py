@@ -32,9 +32,9 @@ from gpu_helpers import assert_ffn_close, bf16_to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-ALL = [mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_AUTO]
+ALL = [mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED, mm.FFN_AUTO]
 NAMES = {mm.FFN_FMA: "fma", mm.FFN_TENSOR_F8: "mxf8f6f4", mm.FFN_TENSOR_F4: "mxf4",
-         mm.FFN_AUTO: "auto"}
+         mm.FFN_TENSOR_FUSED: "fused", mm.FFN_AUTO: "auto"}
 
 
 @pytest.fixture(autouse=True)

@@ -168,7 +168,7 @@ def test_quantize_random_bit_exact(R, K, sd):
     ragged last CTA."""
     key = synth.stream_key(R * 7 + K, "w13_codes")
     z = synth.normal_np(key, 0, R * K).reshape(R, K)
-    row = np.exp2(synth.int_range_np(key, 0, R, -8, 8)).reshape(R, 1)
+    row = np.exp2(synth.int_range_np(key, 0, R, 0, 16) - 8.0).reshape(R, 1)
     _quantize_check(_bf16_bits(z * row * sd), f"R={R} K={K}")
 
 

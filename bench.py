@@ -95,21 +95,27 @@ def kernel_source_tag():
     return h.hexdigest()[:16]
 
 
-def load_traffic(workload, variant_name):
-    """DRAM bytes per FFN call from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
-    p = os.path.join(ROOT, "profiles", f"ffn_{variant_name}_{workload}_traffic.txt")
+def _profile_value(fname, key):
+    """A `key: value` line of a committed ncu summary in profiles/, if the
+    summary was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", fname)
     try:
         kv = {}
         for line in open(p):
-            if ":" in line and not line.startswith("#"):
+            if ":" in line and not line.startswith(("#", "|", " ")):
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
         if kv.get("source_tag") != kernel_source_tag():
             return None
-        return float(kv["dram_bytes_per_ffn_call"])
+        return float(kv[key])
     except Exception:
         return None
+
+
+def load_traffic(workload, variant_name):
+    """DRAM bytes per FFN call from the committed ncu summary (None if it was
+    taken on other kernel sources)."""
+    return _profile_value(f"ffn_{variant_name}_{workload}_traffic.txt", "dram_bytes_per_ffn_call")
 
 
 def workload_config(sh, world):
@@ -678,7 +684,8 @@ def measure_quantize(device, peaks, reps=10):
     return {"kernel": "mxfp4_quantize_kernel", "shape": [R, K], "ms": ms,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": byts,
-                         "traffic": None}}
+                         "traffic": _profile_value("mxfp4_quantize_traffic.md",
+                                                   "dram_bytes_per_launch")}}
 
 
 # --------------------------------------------------------------- per config --

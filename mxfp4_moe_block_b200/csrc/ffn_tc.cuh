@@ -24,7 +24,8 @@
 //   warp 2     TMEM allocation and the single MMA-issuing thread;
 //   warp 3     constant B block scales (kind::mxf4);
 //   warps 4-7  epilogue: TMEM -> registers -> SwiGLU (GEMM-1) or y (GEMM-2);
-//   warps 8-11 scale writers: tcgen05.st of the stage's scale factors;
+//   warps 8-11 scale writers: tcgen05.st of the stage's scale factors
+//              (weights, and kind::mxf8f6f4's activation block scales);
 //   warps 12-15 a second epilogue group (kind::mxf8f6f4).
 // Every wait is bounded; on time-out the kernel records MOE_DEV_TIMEOUT,
 // drains what it issued, frees its TMEM and returns.
@@ -1078,7 +1079,6 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       // more per MMA than the instruction itself.
       const uint64_t a_desc0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
       const uint64_t b_desc0 = smem_desc(smem_u32(smem + C::kOffB), 16, 1024, kSwizzle128B);
-      const uint64_t sfb_desc0 = smem_desc(smem_u32(smem + C::kOffSfb), 0, 128, kSwizzleNone);
       int it = 0;
       for (int t = ring_read(ring_full, ring_empty, ring, it, true, abort, n_tiles);
            t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, true, abort, n_tiles)) {
@@ -1098,24 +1098,13 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         for (int kt = 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&full[stage], phase, abort)) { ok = false; break; }
           // The full barrier completes once the stage's TMA bytes have landed
-          // and the writer warps have stored its A scales into tensor memory
-          // (tcgen05.wait::st + fence before their arrive).  kind::mxf8f6f4's B
-          // block scales reached shared memory by cp.async before the writers
-          // saw them; as in CUTLASS's cp.async-fed UMMA pipelines, the barrier
-          // wait is the only ordering tcgen05.cp needs.
+          // and the writer warps have stored its scale factors into tensor
+          // memory (tcgen05.wait::st + fence before their arrive).
           tc_fence_after();
-          // TMEM: per stage, the A scale groups then, per group, the B row chunks
+          // TMEM: per stage, the A scale groups then, per group, the B row
+          // chunks (all written by the scale-writer warps)
           const uint32_t sfa_t = tmem + sf_col0 + stage * C::kSfCols;
           const uint32_t sfb_t = sfa_t + 4 * Kd::kKGroups;
-          const uint64_t sfb_d = sfb_desc0 + (uint64_t)((stage * C::kSfb) >> 4);
-#pragma unroll
-          for (int g = 0; g < Kd::kKGroups; ++g) {
-            if (!Kd::kRowScaledB)
-#pragma unroll
-            for (int c = 0; c < C::kRowChunks; ++c)
-              tc_cp_32x128b(sfb_t + 4 * (g * C::kRowChunks + c),
-                            sfb_d + (uint64_t)(32 * (g * C::kRowChunks + c)));
-          }
           const uint64_t ad = a_desc0 + (uint64_t)((stage * C::kA) >> 4);
           const uint64_t bd = b_desc0 + (uint64_t)((stage * C::kB) >> 4);
 #pragma unroll
@@ -1151,10 +1140,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       mbar_wait_drain(drain_bar, 0);
     }
   } else if (warp >= 8 && warp < 12) {
-    // ------------------------------------------------- A-scale writers --
-    // Warp 8+q stores lane quarter q of every stage's A scale columns with
-    // tcgen05.st (the scale-factor layout repeats the same 32 lanes in all
-    // four quarters), keeping the copies off the MMA issue path.  Column
+    // --------------------------------------------------- scale writers --
+    // Warp 8+q stores lane quarter q of every stage's scale-factor columns
+    // with tcgen05.st (the scale-factor layout repeats the same 32 lanes in
+    // all four quarters), keeping the copies off the MMA issue path: the A
+    // (weight) scales and, for kind::mxf8f6f4, the B block scales.  Column
     // 4g + j, lane l = the 4 scale bytes of tile row 32j + l, K-group g: the
     // 16 bytes the scale loader put at 512g + 16l.
     // Each leave-or-stay decision is taken by the whole warp (__all_sync):
@@ -1186,6 +1176,18 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           const uint4 g0 = src[0];
           const uint32_t r[4] = {g0.x, g0.y, g0.z, g0.w};
           tc_st_x4(dst, r);
+        }
+        if (!Kd::kRowScaledB) {
+          // kind::mxf8f6f4's B block scales: the same layout, one 128-row
+          // chunk of B after another, behind the A scale columns
+          const uint4 *srb =
+              reinterpret_cast<const uint4 *>(smem + C::kOffSfb + stage * C::kSfb) + lane;
+#pragma unroll
+          for (int gc = 0; gc < Kd::kKGroups * C::kRowChunks; ++gc) {
+            const uint4 v = srb[32 * gc];
+            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+            tc_st_x4(dst + 4 * Kd::kKGroups + 4 * gc, r);
+          }
         }
         tc_wait_st();
         tc_fence_before();

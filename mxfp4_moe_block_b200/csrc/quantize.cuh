@@ -7,7 +7,9 @@
 // OCP MX v1.0 conversion: per 32 consecutive elements of a row the shared
 // scale is 2^(floor(log2 amax) - 2) (2 = the largest E2M1 exponent), and each
 // element becomes the nearest E2M1 value of v / scale, ties to the even
-// code, saturating at +-6, its sign kept.
+// code, saturating at +-6, its sign kept -- the hardware conversion
+// (cvt.rn.satfinite.e2m1x2.f32) applies exactly that rule to the exactly
+// scaled value.
 //
 // HBM-bound: 2 bytes read and 17/32 byte written per element.  Each thread
 // takes 8 consecutive elements (one 16-byte load, one 4-byte store of codes);
@@ -18,17 +20,6 @@
 namespace moe {
 
 constexpr int QUANT_THREADS = 256;
-
-// E2M1 magnitude index (0..7 for 0, .5, 1, 1.5, 2, 3, 4, 6) nearest to a >= 0,
-// ties to the even index, a > 6 saturating at 7.  The midpoints between
-// neighbours are .25 .75 1.25 1.75 2.5 3.5 5; at a midpoint the comparison
-// is strict where the lower neighbour is even and inclusive where the upper
-// one is.
-__device__ __forceinline__ uint32_t e2m1_nearest_even(float a) {
-  return (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
-         (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) +
-         (uint32_t)(a > 5.0f);
-}
 
 // Quantise one group of 8 bf16 (w4 = its 16 bytes) of a 32-element block
 // whose other three groups sit in lanes lane^1, lane^2, lane^3: returns the
@@ -48,15 +39,18 @@ __device__ __forceinline__ uint32_t quantize_group8(const uint4 v, uint32_t *sb)
   const int be = (int)(m >> 7);
   const uint32_t s = (uint32_t)max(0, be - 2);
   const float inv = __uint_as_float((254u - s) << 23);   // 2^(127 - s), exact
+  // v * 2^(127 - s) is exact wherever it can reach 0.25 (and stays below 8);
+  // the conversion rounds it to the nearest E2M1 value, ties to the even
+  // code (the IEEE rule: mantissa bit 0), saturating at +-6 and keeping the
+  // sign (-0 -> code 8); two codes per instruction, the first in the low
+  // nibble
   uint32_t word = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t b = (i & 1) ? (wd[i >> 1] >> 16) : (wd[i >> 1] & 0xffffu);
-    // |v| * 2^(127 - s) is exact wherever it can reach 0.25 (no overflow:
-    // it stays below 8)
-    const float a = __uint_as_float((b & 0x7fffu) << 16) * inv;
-    const uint32_t c = e2m1_nearest_even(a) | ((b >> 12) & 8u);   // sign -> bit 3
-    word |= c << (4 * i);
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = make_float2(bf16_lo(wd[i]) * inv, bf16_hi(wd[i]) * inv);
+    const uint32_t byte =
+        (uint32_t)__nv_cvt_float2_to_fp4x2(f, __NV_E2M1, cudaRoundNearest) & 0xffu;
+    word |= byte << (8 * i);
   }
   *sb = s;
   return word;

@@ -430,7 +430,8 @@ def roofline(wl, ffn_ms, peaks, variant_name):
             "peak": hbm["peak_gbs"] if bound == "hbm" else tc["peak_tflops"],
             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
             "frac": max(t_hbm, t_tc) / ms, "traffic": traffic,
-            "kernel": "mxfp4_moe_ffn (encode, GEMM-1+SwiGLU, encode, GEMM-2 launches)",
+            "kernel": "mxfp4_moe_ffn (every launch of one FFN call: activation encodes and the "
+                      "expert GEMMs, fused or GEMM-1+SwiGLU then GEMM-2)",
             "ffn_ms": ms, "hbm": hbm, "tensor": tc,
             "peak_source": f"{peaks['source']} hbm_gbs / bf16_tflops"}
 

@@ -165,7 +165,8 @@ enum {
   MOE_FFN_TENSOR = 2,    /* tcgen05 block-scaled MMA: TENSOR_F4 while its B
                             tiles stay narrow (8*T*k <= 128 * min(T*k, E)) and
                             H, I are multiples of 256 up to 8192, else
-                            TENSOR_F8                                             */
+                            TENSOR_F8; with a few tokens per expert (B tiles of
+                            at most 32 columns) and I <= 4096, TENSOR_FUSED     */
   MOE_FFN_TENSOR_F8 = 3, /* kind::mxf8f6f4: padded E2M1 weights x two E4M3
                             activation terms with E8M0 block scales               */
   MOE_FFN_TENSOR_F4 = 4, /* kind::mxf4: packed E2M1 weights x eight E2M1

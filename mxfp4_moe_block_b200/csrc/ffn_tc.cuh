@@ -736,8 +736,12 @@ __device__ __forceinline__ int ring_read(uint64_t *ring_full, uint64_t *ring_emp
 // before loading its B operand.  Every CTA is resident at once (one per SM)
 // and tiles are taken in increasing order, so every GEMM-1 tile a waiting
 // GEMM-2 tile needs is held by a running CTA.
+// Register budget: the compiler's own choice for the two GEMMs (no
+// minimum-blocks hint, which let it take up to 168); at most 136 for the
+// fused launch, so that the x encoder's CTAs (256 threads x 48 registers)
+// stay resident beside a GEMM CTA under programmatic dependent launch.
 template <int KIND, int MODE, int BN>
-__global__ void __launch_bounds__(TcKindCfg<KIND>::kThreads, 1)
+__global__ void __launch_bounds__(TcKindCfg<KIND>::kThreads) __maxnreg__(MODE == 3 ? 136 : 168)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcArgs a,
                const __grid_constant__ TcMaps maps2, const __grid_constant__ TcArgs a2) {
   using C = TcCfg<KIND, BN>;
@@ -1572,8 +1576,13 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  int st = FUSED ? tc_attributes<KIND, 3, BN>(dev) : tc_attributes<KIND, 1, BN>(dev);
-  if (st == MOE_OK && !FUSED) st = tc_attributes<KIND, 2, BN>(dev);
+  int st;
+  if constexpr (FUSED) {
+    st = tc_attributes<KIND, 3, BN>(dev);
+  } else {
+    st = tc_attributes<KIND, 1, BN>(dev);
+    if (st == MOE_OK) st = tc_attributes<KIND, 2, BN>(dev);
+  }
   if (st != MOE_OK) return st;
 
   // GEMM-1 (a1): W13 [E*2I, H] x x-terms [T*P, H] -> h; GEMM-2 (a2): W2 [E*H, I]
@@ -1635,7 +1644,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
   }
 
-  if (FUSED) {
+  if constexpr (FUSED) {
     if (launch_pdl(tc_gemm_kernel<KIND, 3, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a1, maps2,
                    a2) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -1654,15 +1663,22 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   return MOE_OK;
 }
 
-template <int KIND, bool FUSED>
-inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
+// B-tile width wanted for a problem: room for the busier experts (1.5 x
+// the average B rows per active expert), and at least 4 tokens.
+template <int KIND>
+inline size_t tc_want(const FfnArgs &f) {
   const size_t P = (size_t)f.T * f.k;
   const size_t used = P < (size_t)f.E ? P : (size_t)f.E;
   const size_t terms = TcKindCfg<KIND>::kTerms;
   const size_t rows = (terms * P + used - 1) / used;           // B rows per expert, average
-  // room for the busier experts, and at least 4 tokens per B tile
   size_t want = rows + rows / 2;
   if (want < 4 * terms) want = 4 * terms;
+  return want;
+}
+
+template <int KIND, bool FUSED>
+inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
+  const size_t want = tc_want<KIND>(f);
   if (want <= 16) return tc_run<KIND, 16, FUSED>(f, ws, sms, s);
   if (want <= 32) return tc_run<KIND, 32, FUSED>(f, ws, sms, s);
   if (want <= 64) return tc_run<KIND, 64, FUSED>(f, ws, sms, s);
@@ -1687,6 +1703,13 @@ inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int ki
                        f.H <= 2 * ENC_THREADS * ENC_MAX_PAIRS &&
                        f.I <= 2 * ENC_THREADS * ENC_MAX_PAIRS;
     kind = (f4_ok && narrow) ? KIND_F4 : KIND_F8;
+    // A few tokens per expert (B tiles of at most 32 columns, as in a
+    // batch-1 block): both GEMMs in one launch, which saves the h encoder's
+    // launch and GEMM-2's ramp (measured 193 vs 200 us at batch 1).  With
+    // wider tiles the fused launch's h encoding -- one warp group of the CTA
+    // that finishes a B tile -- costs more than it saves (4-6 % slower).
+    if (kind == KIND_F4 && tc_want<KIND_F4>(f) <= 32 && f.I <= 2 * 128 * GRP_ENC_MAX_PAIRS)
+      kind = KIND_F4_FUSED;
   }
   if (kind == KIND_F4 || kind == KIND_F4_FUSED) {
     if (f.H % 256 || f.I % 256 || f.H > 2 * ENC_THREADS * ENC_MAX_PAIRS ||

@@ -172,7 +172,7 @@ enum {
   MOE_FFN_TENSOR_F4 = 4, /* kind::mxf4: packed E2M1 weights x eight E2M1
                             activation terms with one scale per row and term
                             (H, I multiples of 256, at most 8192)                 */
-  MOE_FFN_TENSOR_FUSED = 5 /* TENSOR_F4 with both GEMMs in one persistent
+  MOE_FFN_TENSOR_FUSED = 5, /* TENSOR_F4 with both GEMMs in one persistent
                             launch (I <= 4096): the last GEMM-1 tile of each
                             expert's token block encodes its h rows and
                             publishes them by a flag, and GEMM-2 tiles wait
@@ -180,6 +180,12 @@ enum {
                             of a launch -- the first piece of a persistent
                             verify kernel, after the persistent engine of
                             [P4] (prior art).  Same results as TENSOR_F4.   */
+  MOE_FFN_TENSOR_F8_PAIR = 6 /* TENSOR_F8 on clusters of two CTAs (H a multiple
+                            of 256): each M = 256 tcgen05 MMA (cta_group::2)
+                            covers two weight m-blocks, each SM of the pair
+                            holding one m-block and half of the activation
+                            rows, so an SM streams half the activation bytes
+                            per weight byte.  Same results as TENSOR_F8.    */
 };
 /* Accuracy domain of the activation encodings.  FMA and TENSOR_F8 represent
  * every 32-element block of an activation row on its own scale, so they meet

@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(HERE, "libmxfp4_moe.so")
 MOE_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
                 4: "workspace", 5: "device status"}
-FFN_AUTO, FFN_FMA, FFN_TENSOR, FFN_TENSOR_F8, FFN_TENSOR_F4, FFN_TENSOR_FUSED = 0, 1, 2, 3, 4, 5
+(FFN_AUTO, FFN_FMA, FFN_TENSOR, FFN_TENSOR_F8, FFN_TENSOR_F4, FFN_TENSOR_FUSED,
+ FFN_TENSOR_F8_PAIR) = 0, 1, 2, 3, 4, 5, 6
 
 _c_int, _c_float, _c_size, _vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
 

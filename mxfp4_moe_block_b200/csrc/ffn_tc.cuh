@@ -31,6 +31,7 @@
 // drains what it issued, frees its TMEM and returns.
 #pragma once
 #include <cuda.h>
+#include <atomic>
 #include <mutex>
 #include "common.cuh"
 #include "ffn_fma.cuh"
@@ -132,6 +133,15 @@ __device__ __forceinline__ float ld_weak_f32(const float *p) {
   asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
   return v;
 }
+// 16 bytes through the coherent path (rows this CTA wrote in this launch)
+__device__ __forceinline__ uint4 ld_global_v4(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_release_gpu(int *p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -161,6 +171,37 @@ __device__ __noinline__ bool wait_flag(const int *f, volatile int *abort) {
 __device__ __forceinline__ bool mbar_wait_fast(uint64_t *bar, uint32_t parity,
                                                volatile int *abort) {
   return mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort);
+}
+
+// The same with acquire at cluster scope: barriers that the other CTA of a
+// pair arrives on (release at cluster scope).
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __noinline__ bool mbar_wait_cl(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  const uint64_t t0 = global_ns();
+  const uint64_t limit = *(volatile unsigned long long *)&g_wait_limit_ns;
+  for (;;) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 >= limit) {
+      raise_status(MOE_DEV_TIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_fast_cl(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort) {
+  return mbar_try_wait_cl(bar, parity) || mbar_wait_cl(bar, parity, abort);
 }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1,
@@ -215,9 +256,9 @@ constexpr uint32_t kSwizzle128B = 2, kSwizzleNone = 0;
 // K-major A and B: a/b formats (mxf8f6f4: 5 = E2M1, 0 = E4M3; mxf4: 1 =
 // E2M1), N, and the byte of the scale word each operand's scales start at.
 __device__ __forceinline__ uint32_t idesc_block_scaled(uint32_t afmt, uint32_t bfmt, int n,
-                                                       uint32_t sf_id) {
+                                                       uint32_t sf_id, uint32_t m = 128) {
   return (sf_id << 4) | (afmt << 7) | (bfmt << 10) | ((uint32_t)(n >> 3) << 17) | (1u << 23) |
-         ((128u >> 4) << 24) | (sf_id << 29);
+         ((m >> 4) << 24) | (sf_id << 29);
 }
 
 __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -251,6 +292,62 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+
+// ---- CTA pairs (tcgen05 cta_group::2): one M = 256 MMA over two SMs ----
+// The even CTA of a cluster of two issues the MMAs; each CTA holds its own
+// 128 weight rows, half of the B rows and, in its tensor memory, its rows'
+// accumulators (every column) and scale factors (A: its rows; B: all rows).
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate));
+}
+// completion of the pair's MMAs, signalled on the barrier at the same offset
+// in both CTAs
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_rank(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on the other CTA's barrier.  The default semantics (release at CTA
+// scope): the signal only orders this thread's completed tensor-memory
+// stores and barrier waits, and a cluster-scope release measured ~0.9 us per
+// arrive, stalling the pipeline.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// every thread of both CTAs
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
 }
 
 // 32 lanes x 16 columns of 32-bit accumulator -> 16 registers per thread;
@@ -387,7 +484,7 @@ __device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t
 
 // Kind of tensor-core MMA used by the FFN (KIND_F4_FUSED: kind::mxf4, both
 // GEMMs in one launch -- a host-side choice only; the kernels see KIND_F4).
-enum TcKind { KIND_F8 = 0, KIND_F4 = 1, KIND_F4_FUSED = 2 };
+enum TcKind { KIND_F8 = 0, KIND_F4 = 1, KIND_F4_FUSED = 2, KIND_F8_PAIR = 3 };
 constexpr int kF4Terms = 8;     // E2M1 terms per activation row (kind::mxf4)
 
 template <int KIND>
@@ -405,6 +502,49 @@ struct TcKindCfg {
   static constexpr int kRingReaders = 1 + 1 + 4 * kEpiGroups + 4;
   static constexpr bool kRowScaledB = KIND == KIND_F4;          // B scales per row, not block
 };
+
+// Four E4M3 codes (the first in the lowest byte) and back: the paired
+// hardware conversions, round to nearest even, saturating.
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xffffu) | ((hi & 0xffffu) << 16);
+}
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<const __half2 *>(&h));
+}
+
+// One whole 32-element block of an activation row, held by one thread: its
+// two E4M3 terms (32 code bytes each, written as two 16-byte stores to q0 and
+// q1) and their scale bytes -- the encoding of encode_e4m3x2, with the block
+// maximum taken over the thread's own values instead of across a warp.
+__device__ __forceinline__ void encode_block_f8(float (&v)[32], uint8_t *q0, uint8_t *q1,
+                                                uint8_t *s0, uint8_t *s1) {
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    uint32_t mb = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mb = max(mb, __float_as_uint(fabsf(v[e])));
+    const float amax = __uint_as_float(mb);
+    const int s = amax > 0.f ? e4m3_block_exp(amax) : 0;
+    const float inv = pow2f(-s), sc = pow2f(s);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w[i] = e4m3x4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+      const float2 lo = e4m3x2_to_f32(w[i]), hi = e4m3x2_to_f32(w[i] >> 16);
+      v[4 * i] -= lo.x * sc;
+      v[4 * i + 1] -= lo.y * sc;
+      v[4 * i + 2] -= hi.x * sc;
+      v[4 * i + 3] -= hi.y * sc;
+    }
+    uint4 *q = reinterpret_cast<uint4 *>(t ? q1 : q0);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    *(t ? s1 : s0) = (uint8_t)(127 + s);
+  }
+}
 
 // Stores one lane's two E4M3 terms of element n of activation row r (B rows
 // 2r, 2r+1) and, from lane 0, the block's two scale bytes.
@@ -662,20 +802,29 @@ struct TcArgs {
 
 constexpr int kMaxStages = 12;
 
-template <int KIND, int BN>
+// PAIR: the stage holds this CTA's half of the B rows (the other CTA of the
+// pair holds the other half).
+template <int KIND, int BN, int PAIR = 0>
 struct TcCfg {
   using Kd = TcKindCfg<KIND>;
   static constexpr int kRowChunks = (BN + 127) / 128;               // 128-row scale chunks of B
   static constexpr int kA = 128 * 128;                              // smem bytes of one A stage
-  static constexpr int kB = BN * 128;
+  static constexpr int kB = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kSfa = 512 * Kd::kKGroups;
   static constexpr int kSfb = Kd::kRowScaledB ? 0 : 512 * Kd::kKGroups * kRowChunks;
   static constexpr int kSfbConst = Kd::kRowScaledB ? 512 * kRowChunks : 0;  // all 1.0
-  static constexpr int kStageBytes = kA + kB + kSfa + kSfb;
+  // kind::mxf8f6f4: the scale bytes have a ring of their own, refilled as
+  // soon as the writer warps have moved a slot into tensor memory (not when
+  // the MMAs release the stage), so the scale loads run that much further
+  // ahead; sized to leave the operand stages as many as before.  Else one
+  // scale slot per operand stage.
+  static constexpr int kSfRing = KIND == KIND_F8 ? (PAIR ? 8 : 4) : 0;
+  static constexpr int kStageBytes = kA + kB + (kSfRing ? 0 : kSfa + kSfb);
   static constexpr int kFixed = 1024 + Kd::kEpiGroups * 64 * (16 / Kd::kTerms) * 4 + 1026 * 2 +
                                  2 * 1025 * 4 + 128 + 1024 + kSfbConst;
-  static constexpr int kStages0 = (227 * 1024 - kFixed) / kStageBytes;
+  static constexpr int kStages0 = (227 * 1024 - kFixed - kSfRing * (kSfa + kSfb)) / kStageBytes;
   static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
+  static constexpr int kSfSlots = kSfRing ? kSfRing : kStages;
   static constexpr int kSfCols =                                    // TMEM columns per stage
       4 * Kd::kKGroups * (Kd::kRowScaledB ? 1 : 1 + kRowChunks);
   // Independent accumulation chains per buffer: with few B columns each MMA
@@ -693,8 +842,8 @@ struct TcCfg {
   static_assert(kUsed <= 512, "TMEM budget");
   static constexpr int kOffB = kStages * kA;
   static constexpr int kOffSfa = kOffB + kStages * kB;
-  static constexpr int kOffSfb = kOffSfa + kStages * kSfa;
-  static constexpr int kOffBar = kOffSfb + kStages * kSfb;
+  static constexpr int kOffSfb = kOffSfa + kSfSlots * kSfa;
+  static constexpr int kOffBar = kOffSfb + kSfSlots * kSfb;
   // SwiGLU exchange: 64 rows x (tokens per 16-column chunk) floats per
   // epilogue warp group
   static constexpr int kXchgFloats = 64 * (16 / Kd::kTerms);
@@ -740,11 +889,19 @@ __device__ __forceinline__ int ring_read(uint64_t *ring_full, uint64_t *ring_emp
 // minimum-blocks hint, which let it take up to 168); at most 136 for the
 // fused launch, so that the x encoder's CTAs (256 threads x 48 registers)
 // stay resident beside a GEMM CTA under programmatic dependent launch.
-template <int KIND, int MODE, int BN>
+// PAIR (kind::mxf8f6f4, MODES 1 and 2): clusters of two CTAs, each tile two
+// m-blocks of one B tile -- rank r of the pair takes m-block 2m + r and half
+// of the B rows; the even CTA issues M = 256 MMAs (cta_group::2) over both.
+// Each CTA's own loads complete on its own full barrier; its scale writers
+// then tell the even CTA (ready), whose MMAs release both CTAs' stages and
+// accumulators with multicast commits.  Tiles are dealt out statically, pair
+// p taking p, p + pairs, ...
+template <int KIND, int MODE, int BN, int PAIR = 0>
 __global__ void __launch_bounds__(TcKindCfg<KIND>::kThreads) __maxnreg__(MODE == 3 ? 136 : 168)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcArgs a,
                const __grid_constant__ TcMaps maps2, const __grid_constant__ TcArgs a2) {
-  using C = TcCfg<KIND, BN>;
+  static_assert(!PAIR || (KIND == KIND_F8 && MODE != 3 && BN >= 64), "CTA pairs: mxf8f6f4 GEMMs");
+  using C = TcCfg<KIND, BN, PAIR>;
   using Kd = TcKindCfg<KIND>;
   constexpr int T = Kd::kTerms;
   extern __shared__ uint8_t smem_raw[];
@@ -755,16 +912,22 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   uint64_t *acc_empty = acc_full + 2;          // [2]
   volatile int *abort = reinterpret_cast<volatile int *>(acc_empty + 2);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 3);
-  uint64_t *sfs_full = acc_empty + 4;          // [kStages] scale bytes landed in smem
+  uint64_t *sfs_full = acc_empty + 4;          // [kSfSlots] scale bytes landed in smem
   // tile ring: the producer publishes each tile index it takes; every other
   // role reads the same sequence
-  uint64_t *ring_full = sfs_full + C::kStages;  // [kRing]
+  uint64_t *ring_full = sfs_full + C::kSfSlots;  // [kRing]
   uint64_t *ring_empty = ring_full + kRing;     // [kRing]
   volatile int *ring = reinterpret_cast<volatile int *>(ring_empty + kRing);   // [kRing]
   // end of the kernel: the MMA thread's last commit, and the number of
   // stages the producer issued (the abort path drains them)
   uint64_t *drain_bar = ring_empty + kRing + 2;
   volatile int *s_issued = reinterpret_cast<volatile int *>(drain_bar + 1);
+  // PAIR, even CTA: a stage's operands and scale factors are in place in
+  // both CTAs (the 4 + 4 scale-writer warps)
+  uint64_t *ready = drain_bar + 2;              // [kStages]
+  // kSfRing: a scale slot moved to tensor memory (4 writer warps)
+  uint64_t *sfs_empty = ready + C::kStages;     // [kSfSlots]
+  static_assert(8 * (3 * C::kStages + 2 * C::kSfSlots + 2 * kRing + 10) <= 960, "barrier region");
   float *xchg = reinterpret_cast<float *>(smem + C::kOffXchg);
   // The table stays small: a GEMM CTA leaves a few KB of the SM's shared
   // memory free, so that the encode kernels' CTAs can become resident beside
@@ -774,16 +937,21 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   int *s_r0 = s_pre + 1025;        // first sorted row of each active expert (+ total)
 
   // the fused FFN's encode scratch: the last-tile flag and the row maxima
-  volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::kOffBar + 512);
-  float *s_red = reinterpret_cast<float *>(smem + C::kOffBar + 512 + 16);
+  volatile int *s_last = reinterpret_cast<volatile int *>(smem + C::kOffBar + 960);
+  float *s_red = reinterpret_cast<float *>(smem + C::kOffBar + 960 + 16);   // [8]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t crank = PAIR ? cluster_rank() : 0u;   // rank in the pair
+  const bool leader = crank == 0;
+  const int pair_id = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   // m-blocks of a B tile and K stages, per phase (phase 1: MODE 3 only)
   const int mt1 = MODE == 2 ? a.rows_per_expert / 128 : a.I / 64;
   const int mt2 = a2.rows_per_expert / 128;
   const int ks1 = a.K / Kd::kStageK, ks2 = a2.K / Kd::kStageK;
-  // the table's prefix is in tiles (MODES 1, 2) or in B tiles (MODE 3)
-  const int mtiles = MODE == 3 ? 1 : mt1;
+  // the table's prefix is in tiles (MODES 1, 2; PAIR: tiles of two
+  // m-blocks) or in B tiles (MODE 3)
+  const int mtiles = MODE == 3 ? 1 : PAIR ? mt1 / 2 : mt1;
 
   // tile table: active experts and the prefix of their tile counts
   if (warp == 0) {
@@ -817,9 +985,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     }
   } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1 + 4);      // producer expect_tx + 4 A-scale writer warps
+      // producer expect_tx + 4 A-scale writer warps (PAIR: the producer's
+      // expect_tx alone; the writers report to the even CTA's ready)
+      mbar_init(&full[s], PAIR ? 1 : 1 + 4);
       mbar_init(&empty[s], 1);         // MMA commit
+      if (PAIR) mbar_init(&ready[s], 8);
+    }
+    for (int s = 0; s < C::kSfSlots; ++s) {
       mbar_init(&sfs_full[s], 32);     // 32 scale-loader lanes (cp.async)
+      if (C::kSfRing) mbar_init(&sfs_empty[s], 4);   // 4 scale-writer warps
     }
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&ring_full[r], 1);             // producer
@@ -827,17 +1001,26 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4 * Kd::kEpiGroups);   // one arrival per epilogue warp
+      // one arrival per epilogue warp (PAIR: of both CTAs)
+      mbar_init(&acc_empty[b], (PAIR ? 8 : 4) * Kd::kEpiGroups);
     }
     mbar_init(drain_bar, 1);           // the MMA thread's final commit
     *abort = 0;
     *s_issued = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   } else if (warp == 2) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(C::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if (PAIR) {
+      // both CTAs' warp 2: the same columns in each CTA's tensor memory
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
   }
   if (Kd::kRowScaledB && warp == 3) {
     // constant B block scales (byte 127 = 1.0), copied to tensor memory once
@@ -847,6 +1030,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   }
   tc_fence_before();
   __syncthreads();
+  // a pair's barriers are initialised before either CTA signals the other's
+  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_act = s_act[1024];
@@ -882,7 +1067,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     const int ne = s_r0[lo + 1] - r0;
     const int nt_cnt = (T * ne + BN - 1) / BN;
     const int local = tl - s_pre[lo] * mtl;
-    r.mt = local / nt_cnt;
+    r.mt = PAIR ? 2 * (local / nt_cnt) + (int)crank : local / nt_cnt;
     const int nt = local % nt_cnt;
     r.g = s_pre[lo] + nt;
     r.rowB = T * r0 + nt * BN;
@@ -904,11 +1089,19 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       // loads at most 15 rows more than the tile's N.  bsel = box class
       // (0..3) | (class of the second box + 1) << 3.
       auto box_class = [](int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; };
+      // PAIR: N rounded up to 32, this CTA's half (a multiple of 16 rows)
+      // in one box of up to 64 rows or a 64-row box and a second one.
       auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel, int &ph, int &g) {
         const Tile tl = decode(t);
-        const int ncol = (tl.nB + 15) & ~15;
-        bsel = ncol <= 128 ? box_class(ncol) : 3 | ((box_class(ncol - 128) + 1) << 3);
-        rowB = tl.rowB;
+        if (PAIR) {
+          const int half = ((tl.nB + 31) & ~31) / 2;
+          bsel = half <= 64 ? box_class(half) : 2 | ((box_class(half - 64) + 1) << 3);
+          rowB = tl.rowB + (int)crank * half;
+        } else {
+          const int ncol = (tl.nB + 15) & ~15;
+          bsel = ncol <= 128 ? box_class(ncol) : 3 | ((box_class(ncol - 128) + 1) << 3);
+          rowB = tl.rowB;
+        }
         ph = tl.ph;
         g = tl.g;
         const int rpe = ph ? a2.rows_per_expert : a.rows_per_expert;
@@ -931,9 +1124,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       auto load_b = [&](int st, int bsel, int rowB, int kt, int ph) {
         uint8_t *sb = smem + C::kOffB + st * C::kB;
         const CUtensorMap *mb = ph ? maps2.b : maps.b;
+        constexpr int kFirst = PAIR ? 64 : 128;   // rows of the first box when there are two
         tma_load_2d(sb, &mb[bsel & 7], kt * 128, rowB, &full[st], pol_x);
         if (bsel >> 3)
-          tma_load_2d(sb + 128 * 128, &mb[(bsel >> 3) - 1], kt * 128, rowB + 128, &full[st],
+          tma_load_2d(sb + kFirst * 128, &mb[(bsel >> 3) - 1], kt * 128, rowB + kFirst, &full[st],
                       pol_x);
       };
       // a GEMM-2 tile of the fused FFN: its B operand (h rows encoded by the
@@ -947,8 +1141,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         return ok;
       };
       // Tile sequence: blockIdx.x first, then gridDim.x + (the counter's next
-      // value) -- a CTA whose tiles went fast takes more.  Each index is
-      // published into the ring as soon as it is known.
+      // value) -- a CTA whose tiles went fast takes more (PAIR: pair p takes
+      // p, p + pairs, ..., the same in both CTAs).  Each index is published
+      // into the ring as soon as it is known.
       int published = 0;
       auto publish = [&](int t) {
         const int slot = published % kRing;
@@ -960,13 +1155,13 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         ++published;
         return true;
       };
-      publish(blockIdx.x);
+      publish(pair_id);
       // Weights depend on no earlier kernel: the first tile's leading stages
       // of A stream in before the wait for the activation operand.
       int npre = 0;
-      if ((int)blockIdx.x < n_tiles) {
+      if (pair_id < n_tiles) {
         int arow, rowB, bsel, ph, g;
-        tile_geom(blockIdx.x, arow, rowB, bsel, ph, g);
+        tile_geom(pair_id, arow, rowB, bsel, ph, g);
         npre = min(C::kStages, ksteps_of(ph));
         for (int kt = 0; kt < npre; ++kt) {
           mbar_expect_tx(&full[kt], Kd::kABytes + b_bytes(bsel));
@@ -983,16 +1178,16 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         pdl_wait();
         pdl_trigger();
       }
-      for (int t = blockIdx.x; t < n_tiles && !*abort;) {
+      for (int t = pair_id; t < n_tiles && !*abort;) {
         // the next tile, published before this one's stages are issued
-        const int t_next = (int)gridDim.x + atomicAdd(a.tile_counter, 1);
+        const int t_next = PAIR ? t + n_units : n_units + atomicAdd(a.tile_counter, 1);
         if (!publish(t_next < n_tiles ? t_next : n_tiles)) break;
         int arow, rowB, bsel, ph, g;
         tile_geom(t, arow, rowB, bsel, ph, g);
         const uint32_t bbytes = b_bytes(bsel);
-        if (t != (int)blockIdx.x && !b_ready(ph, g)) break;
+        if (t != pair_id && !b_ready(ph, g)) break;
         const int ksteps = ksteps_of(ph);
-        for (int kt = t == (int)blockIdx.x ? npre : 0; kt < ksteps; ++kt) {
+        for (int kt = t == pair_id ? npre : 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
           load_a(stage, arow, kt, ph);
@@ -1036,7 +1231,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       }
       const int ksteps = ksteps_of(tl.ph);
       for (int kt = 0; kt < ksteps; ++kt) {
-        if (!__all_sync(FULL, mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
+        // the slot is free: its last bytes are in tensor memory (kSfRing), or
+        // the MMAs that read its stage's columns are done
+        if (!__all_sync(FULL, C::kSfRing ? mbar_wait_fast(&sfs_empty[stage], phase ^ 1, abort)
+                                         : mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
           ok = false;
           break;
         }
@@ -1058,13 +1256,20 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         }
         cp_async_arrive_noinc(&sfs_full[stage]);
         ++l_signaled;
-        if (++stage == C::kStages) { stage = 0; phase ^= 1; }
+        if (++stage == C::kSfSlots) { stage = 0; phase ^= 1; }
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 2) {
     // ----------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    if (PAIR && !leader && lane == 0) {
+      // the odd CTA of a pair issues no MMAs; it only takes its turn in the
+      // tile ring
+      for (int it = 0;; ++it) {
+        const int t = ring_read(ring_full, ring_empty, ring, it, true, abort, n_tiles);
+        if (t >= n_tiles || *abort) break;
+      }
+    } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       const uint32_t sf_col0 = (uint32_t)C::kAccCols;
@@ -1087,23 +1292,31 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       for (int t = ring_read(ring_full, ring_empty, ring, it, true, abort, n_tiles);
            t < n_tiles && !*abort; t = ring_read(ring_full, ring_empty, ring, ++it, true, abort, n_tiles)) {
         const Tile tl = decode(t);
-        const int ncol = (tl.nB + 15) & ~15;
+        const int ncol = PAIR ? (tl.nB + 31) & ~31 : (tl.nB + 15) & ~15;
         const int ksteps = ksteps_of(tl.ph);
         // the tile's instruction descriptor; MMA kk or-s in its scale byte
         // selector (sf_id, bits 4-5 and 29-30)
-        const uint32_t idesc0 =
-            KIND == KIND_F4 ? idesc_block_scaled(1, 1, ncol, 0) : idesc_block_scaled(5, 0, ncol, 0);
+        const uint32_t idesc0 = KIND == KIND_F4 ? idesc_block_scaled(1, 1, ncol, 0)
+                                                : idesc_block_scaled(5, 0, ncol, 0, PAIR ? 256 : 128);
         const int buf = it % C::kAcc;
         const uint32_t use = (uint32_t)(it / C::kAcc);
-        if (!mbar_wait_fast(&acc_empty[buf], (use & 1) ^ 1, abort)) break;
+        if (!(PAIR ? mbar_wait_fast_cl(&acc_empty[buf], (use & 1) ^ 1, abort)
+                   : mbar_wait_fast(&acc_empty[buf], (use & 1) ^ 1, abort)))
+          break;
         tc_fence_after();
         const uint32_t acc_t = tmem + (uint32_t)(buf * C::kChains * BN);
         bool ok = true;
         for (int kt = 0; kt < ksteps; ++kt) {
-          if (!mbar_wait_fast(&full[stage], phase, abort)) { ok = false; break; }
+          if (!(PAIR ? mbar_wait_fast_cl(&ready[stage], phase, abort)
+                     : mbar_wait_fast(&full[stage], phase, abort))) {
+            ok = false;
+            break;
+          }
           // The full barrier completes once the stage's TMA bytes have landed
           // and the writer warps have stored its scale factors into tensor
-          // memory (tcgen05.wait::st + fence before their arrive).
+          // memory (tcgen05.wait::st + fence before their arrive); PAIR: the
+          // ready barrier, once the writer warps of both CTAs have seen their
+          // CTA's bytes land and stored its scale factors.
           tc_fence_after();
           // TMEM: per stage, the A scale groups then, per group, the B row
           // chunks (all written by the scale-writer warps)
@@ -1125,22 +1338,27 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
                        sfb_const_t | (sfid << 30), acc);
             } else {
               const uint32_t sfid = (uint32_t)kk;
-              mma_mxf8f6f4(d_t, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
-                           idesc0 | (sfid << 4) | (sfid << 29), sfa_t | (sfid << 30),
-                           sfb_t | (sfid << 30), acc);
+              if (PAIR)
+                mma_mxf8f6f4_pair(d_t, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                                  idesc0 | (sfid << 4) | (sfid << 29), sfa_t | (sfid << 30),
+                                  sfb_t | (sfid << 30), acc);
+              else
+                mma_mxf8f6f4(d_t, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk),
+                             idesc0 | (sfid << 4) | (sfid << 29), sfa_t | (sfid << 30),
+                             sfb_t | (sfid << 30), acc);
             }
           }
-          tc_commit(&empty[stage]);
+          if (PAIR) tc_commit_pair_both(&empty[stage]); else tc_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(&acc_full[buf]);
+        if (PAIR) tc_commit_pair_both(&acc_full[buf]); else tc_commit(&acc_full[buf]);
       }
       // Every MMA and tensor-memory copy this thread issued completes before
       // the CTA frees its tensor memory, on every exit path: one more commit
       // tracks them all.  (On the normal path the epilogue has waited for the
       // last tile already, so this costs nothing.)
-      tc_commit(drain_bar);
+      if (PAIR) tc_commit_pair(drain_bar); else tc_commit(drain_bar);
       mbar_wait_drain(drain_bar, 0);
     }
   } else if (warp >= 8 && warp < 12) {
@@ -1157,6 +1375,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int stage = 0;
     uint32_t phase = 0;
+    int slot = 0;          // scale slot (the stage itself unless kSfRing)
+    uint32_t sph = 0;
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
       const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
@@ -1165,12 +1385,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       for (int kt = 0; kt < ksteps; ++kt) {
         // the MMAs that read this stage's columns last time are done, and the
         // stage's scale bytes are in shared memory
-        const bool ready = mbar_wait_fast(&empty[stage], phase ^ 1, abort) &&
-                           mbar_wait_fast(&sfs_full[stage], phase, abort);
-        if (!__all_sync(FULL, ready)) { ok = false; break; }
+        const bool rdy = mbar_wait_fast(&empty[stage], phase ^ 1, abort) &&
+                         mbar_wait_fast(&sfs_full[slot], sph, abort);
+        if (!__all_sync(FULL, rdy)) { ok = false; break; }
         tc_fence_after();
         const uint4 *src =
-            reinterpret_cast<const uint4 *>(smem + C::kOffSfa + stage * C::kSfa) + lane;
+            reinterpret_cast<const uint4 *>(smem + C::kOffSfa + slot * C::kSfa) + lane;
         const uint32_t dst = tmem + lane_base + (uint32_t)C::kAccCols + stage * C::kSfCols;
         if (Kd::kKGroups == 2) {
           const uint4 g0 = src[0], g1 = src[32];
@@ -1185,7 +1405,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           // kind::mxf8f6f4's B block scales: the same layout, one 128-row
           // chunk of B after another, behind the A scale columns
           const uint4 *srb =
-              reinterpret_cast<const uint4 *>(smem + C::kOffSfb + stage * C::kSfb) + lane;
+              reinterpret_cast<const uint4 *>(smem + C::kOffSfb + slot * C::kSfb) + lane;
 #pragma unroll
           for (int gc = 0; gc < Kd::kKGroups * C::kRowChunks; ++gc) {
             const uint4 v = srb[32 * gc];
@@ -1196,7 +1416,25 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
+        if (C::kSfRing) {
+          // the slot's bytes are in registers and stored: the loader may refill it
+          if (lane == 0) mbar_arrive(&sfs_empty[slot]);
+          if (++slot == C::kSfSlots) { slot = 0; sph ^= 1; }
+        } else {
+          slot = stage == C::kStages - 1 ? 0 : stage + 1;
+          sph = stage == C::kStages - 1 ? phase ^ 1 : phase;
+        }
+        if (PAIR) {
+          // this CTA's operand bytes have landed too; then the even CTA hears
+          // of both
+          if (!__all_sync(FULL, mbar_wait_fast(&full[stage], phase, abort))) { ok = false; break; }
+          if (lane == 0) {
+            if (leader) mbar_arrive(&ready[stage]);
+            else mbar_arrive_cluster(mapa_rank(&ready[stage], 0));
+          }
+        } else if (lane == 0) {
+          mbar_arrive(&full[stage]);
+        }
         ++w_arrived;
         if (++stage == C::kStages) { stage = 0; phase ^= 1; }
       }
@@ -1207,6 +1445,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     // groups of four warps (4-7 and 12-15, one per TMEM lane quarter each)
     // take alternate 16-column chunks.
     const int q = warp & 3;                     // TMEM lane quarter
+    // hand an accumulator buffer back to the MMA thread (PAIR: the even CTA's)
+    auto release_acc = [&](int b) {
+      if (PAIR && !leader) mbar_arrive_cluster(mapa_rank(&acc_empty[b], 0));
+      else mbar_arrive(&acc_empty[b]);
+    };
     const int grp = warp >= 12 ? 1 : 0;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     float *gx = xchg + grp * C::kXchgFloats;
@@ -1262,7 +1505,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         // no chunk for this group: hand the buffer back at once
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
       }
       for (int c0 = cfirst; c0 < nB; c0 += 16 * Kd::kEpiGroups) {
         float v[16];
@@ -1285,7 +1528,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           // buffer back to the MMA warp before the arithmetic and the stores
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          if (lane == 0) release_acc(buf);
         }
         const int tok0 = c0 / T;
         float tok_sum[kTokPerLd];
@@ -1321,29 +1564,63 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           // handing the other its half through disjoint slots of xchg.
           const int qq = q & 1;
           const bool gate = q < 2;
+          // Token j = 2 jj + par of the chunk is this warp's (par = 0 for the
+          // gate warp); the loops below have no data-dependent branch, so the
+          // warp's tokens run as independent chains.
           const int slot0 = (32 * qq + lane) * kTokPerLd;
+          const int par = gate ? 0 : 1;
+          constexpr int kOwn = kTokPerLd / 2;
 #pragma unroll
-          for (int j = 0; j < kTokPerLd; ++j)
-            if ((j & 1) == (gate ? 1 : 0)) gx[slot0 + j] = tok_sum[j];
+          for (int jj = 0; jj < kOwn; ++jj)   // the other warp's tokens
+            gx[slot0 + 2 * jj + 1 - par] = gate ? tok_sum[2 * jj + 1] : tok_sum[2 * jj];
           group_sync(grp);
           {
             const int n = mt * 64 + 32 * qq + lane;
 #pragma unroll
-            for (int j = 0; j < kTokPerLd; ++j) {
-              if ((j & 1) != (gate ? 0 : 1)) continue;
-              const int tok = tok0 + j;
-              const float g = gate ? tok_sum[j] : gx[slot0 + j];
-              const float u = gate ? gx[slot0 + j] : tok_sum[j];
-              const uint16_t hb = f32_to_bf16_bits(g / (1.f + expf(-g)) * u);
-              const bool valid = tok < ntok;
-              const size_t r = (size_t)(rtok0 + tok);
-              if (valid) a.h[r * a.I + n] = hb;
-              if (!Kd::kRowScaledB)     // kind::mxf4 encodes h rows in a separate pass
-                store_terms_f8(__uint_as_float((uint32_t)hb << 16), r, n, a.I, a.hq, a.hs,
-                               lane, valid);
+            for (int jj = 0; jj < kOwn; ++jj) {
+              const int j = 2 * jj + par;
+              const float own = gate ? tok_sum[2 * jj] : tok_sum[2 * jj + 1];
+              const float oth = gx[slot0 + j];
+              const float g = gate ? own : oth;
+              const float u = gate ? oth : own;
+              // SiLU(g) * u, rounded to bf16 (the fast exponential and divide
+              // are far inside the bf16 rounding step)
+              const uint16_t hb = f32_to_bf16_bits(__fdividef(g, 1.f + __expf(-g)) * u);
+              if (tok0 + j < ntok) a.h[(size_t)(rtok0 + tok0 + j) * a.I + n] = hb;
             }
           }
           group_sync(grp);
+        }
+      }
+      if (!Kd::kRowScaledB && md == 1) {
+        // kind::mxf8f6f4's GEMM-2 operand: two E4M3 terms of h with a scale
+        // byte per 32-element block.  Each thread takes whole blocks -- one
+        // token's 32 h columns of this tile, read back after the group's
+        // barrier -- of the tokens this group finished: chunk k of the group
+        // held tokens 16k + 8 grp .. +7.
+        group_sync(grp);
+        const int nch = nB > 16 * grp ? (nB - 16 * grp + 31) / 32 : 0;
+        for (int p = 32 * q + lane; p < 16 * nch; p += 128) {
+          const int lt = p >> 1, b = p & 1;
+          const int tok = 16 * (lt >> 3) + 8 * grp + (lt & 7);
+          if (tok >= ntok) continue;
+          const size_t r = (size_t)(rtok0 + tok);
+          const int col = mt * 64 + 32 * b;
+          const uint4 *src = reinterpret_cast<const uint4 *>(a.h + r * a.I + col);
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = ld_global_v4(src + i);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              v[8 * i + 2 * k] = __uint_as_float(ww[k] << 16);
+              v[8 * i + 2 * k + 1] = __uint_as_float(ww[k] & 0xffff0000u);
+            }
+          }
+          encode_block_f8(v, a.hq + (2 * r) * a.I + col, a.hq + (2 * r + 1) * a.I + col,
+                          a.hs + (2 * r) * (a.I / 32) + col / 32,
+                          a.hs + (2 * r + 1) * (a.I / 32) + col / 32);
         }
       }
       if (MODE == 3 && md == 1) {
@@ -1379,11 +1656,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   // those stages' full barriers (the producer issued at most kStages ahead of
   // them), so that each barrier's phase now waits for its TMA bytes alone,
   // and the producer waits (bounded) for the last stages it issued to land
-  // before the CTA's shared memory is released.
+  // before the CTA's shared memory is released.  (PAIR: a full barrier waits
+  // for the producer and its bytes alone already.)
   __syncthreads();
   if (*abort) {
     const int issued = *s_issued;
-    if (warp >= 8 && warp < 12 && lane == 0)
+    if (!PAIR && warp >= 8 && warp < 12 && lane == 0)
       for (int j = w_arrived; j < issued; ++j) mbar_arrive(&full[j % C::kStages]);
     __syncthreads();
     if (warp == 0 && lane == 0)
@@ -1391,11 +1669,22 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         mbar_wait_drain(&full[j % C::kStages], (uint32_t)(j / C::kStages) & 1u);
     // the scale loader's last signals: their cp.async arrivals have landed
     if (warp == 1)
-      for (int j = max(0, l_signaled - C::kStages); j < l_signaled; ++j)
-        mbar_wait_drain(&sfs_full[j % C::kStages], (uint32_t)(j / C::kStages) & 1u);
+      for (int j = max(0, l_signaled - C::kSfSlots); j < l_signaled; ++j)
+        mbar_wait_drain(&sfs_full[j % C::kSfSlots], (uint32_t)(j / C::kSfSlots) & 1u);
     __syncthreads();
   }
-  if (warp == 2) {
+  if (PAIR) {
+    // An abort ends the other CTA's waits at once; then neither CTA leaves
+    // (its barriers and operands are the other's too) before both are done.
+    if (*abort && threadIdx.x == 0) st_cluster_u32(mapa_rank((const void *)abort, crank ^ 1u), 1u);
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 2) {
+      tc_fence_after();
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(C::kTmemCols));
+    }
+  } else if (warp == 2) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(C::kTmemCols));
@@ -1488,21 +1777,54 @@ inline bool make_weight_map(CUtensorMap *m, const uint8_t *codes, uint64_t K, ui
 // instantiation, set once per device; a failed set is reported and retried
 // on the next call.  Guarded by a mutex: host threads may make their first
 // call at the same time.
-template <int KIND, int MODE, int BN>
+template <int KIND, int MODE, int BN, int PAIR = 0>
 inline int tc_attributes(int dev) {
-  using C = TcCfg<KIND, BN>;
+  using C = TcCfg<KIND, BN, PAIR>;
   static std::mutex mu;
   static unsigned long long done = 0;   // one bit per device
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(mu);
   if ((done >> dev) & 1ull) return MOE_OK;
-  if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, MODE, BN>,
+  if (cudaFuncSetAttribute(tc_gemm_kernel<KIND, MODE, BN, PAIR>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   done |= 1ull << dev;
   return MOE_OK;
+}
+
+// CTAs of a paired GEMM launch: two per cluster of two that can be resident
+// at once (a cluster's two SMs sit in one GPC), asked of the runtime once per
+// kernel and process; at most the SM count.
+template <int MODE, int BN>
+inline int tc_pair_grid(int sms) {
+  static std::atomic<int> cached{0};
+  int n = cached.load();
+  if (n == 0) {
+    using C = TcCfg<KIND_F8, BN, 1>;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sms & ~1));
+    cfg.blockDim = dim3(TcKindCfg<KIND_F8>::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, tc_gemm_kernel<KIND_F8, MODE, BN, 1>, &cfg) !=
+            cudaSuccess ||
+        clusters <= 0) {
+      cudaGetLastError();
+      clusters = sms / 2;
+    }
+    n = 2 * std::min(clusters, sms / 2);
+    cached.store(n);
+  }
+  return n;
 }
 
 // The tensor maps of one FFN call depend only on its pointers and sizes;
@@ -1554,11 +1876,13 @@ inline TcMapCache &tc_map_cache() {
 
 // One FFN call on the tensor cores: the x encoder, then GEMM-1 + SwiGLU, the
 // h encoder and GEMM-2 -- or, FUSED (kind::mxf4), the x encoder and one
-// launch of both GEMMs that encodes h itself.
-template <int KIND, int BN, bool FUSED>
+// launch of both GEMMs that encodes h itself; PAIR (kind::mxf8f6f4): both
+// GEMMs on clusters of two CTAs.
+template <int KIND, int BN, bool FUSED, int PAIR = 0>
 int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   static_assert(!FUSED || KIND == KIND_F4, "the fused FFN takes the kind::mxf4 operands");
-  using C = TcCfg<KIND, BN>;
+  static_assert(!PAIR || (KIND == KIND_F8 && !FUSED), "CTA pairs: kind::mxf8f6f4, two launches");
+  using C = TcCfg<KIND, BN, PAIR>;
   using Kd = TcKindCfg<KIND>;
   constexpr int T = Kd::kTerms;
   const size_t P = (size_t)f.T * f.k;
@@ -1580,8 +1904,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   if constexpr (FUSED) {
     st = tc_attributes<KIND, 3, BN>(dev);
   } else {
-    st = tc_attributes<KIND, 1, BN>(dev);
-    if (st == MOE_OK) st = tc_attributes<KIND, 2, BN>(dev);
+    st = tc_attributes<KIND, 1, BN, PAIR>(dev);
+    if (st == MOE_OK) st = tc_attributes<KIND, 2, BN, PAIR>(dev);
   }
   if (st != MOE_OK) return st;
 
@@ -1650,6 +1974,15 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
     return MOE_OK;
   }
+  if constexpr (PAIR != 0) {
+    // clusters of two CTAs, as many as are resident at once
+    if (launch_pdl_cluster(tc_gemm_kernel<KIND, 1, BN, PAIR>, tc_pair_grid<1, BN>(sms),
+                           Kd::kThreads, C::kSmem, 2u, s, maps1, a1, maps1, a1) != cudaSuccess ||
+        launch_pdl_cluster(tc_gemm_kernel<KIND, 2, BN, PAIR>, tc_pair_grid<2, BN>(sms),
+                           Kd::kThreads, C::kSmem, 2u, s, maps2, a2, maps2, a2) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   if (launch_pdl(tc_gemm_kernel<KIND, 1, BN>, sms, Kd::kThreads, C::kSmem, s, maps1, a1, maps1,
                  a1) != cudaSuccess)
     return MOE_ERR_CUDA;
@@ -1687,6 +2020,14 @@ inline int tc_dispatch(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   return tc_run<KIND, 256, FUSED>(f, ws, sms, s);
 }
 
+// kind::mxf8f6f4 on clusters of two CTAs: B tiles of 128, 192 or 256 rows.
+inline int tc_dispatch_pair(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
+  const size_t want = tc_want<KIND_F8>(f);
+  if (want <= 128) return tc_run<KIND_F8, 128, false, 1>(f, ws, sms, s);
+  if (want <= 192) return tc_run<KIND_F8, 192, false, 1>(f, ws, sms, s);
+  return tc_run<KIND_F8, 256, false, 1>(f, ws, sms, s);
+}
+
 // kind::mxf4 (packed FP4 weights, 4 activation terms) when K allows 256-wide
 // stages, else kind::mxf8f6f4.
 inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int kind) {
@@ -1721,6 +2062,11 @@ inline int tc_ffn(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s, int ki
       return tc_dispatch<KIND_F4, true>(f, ws, sms, s);
     }
     return tc_dispatch<KIND_F4, false>(f, ws, sms, s);
+  }
+  if (kind == KIND_F8_PAIR) {
+    // GEMM-2's m-blocks (H / 128 of them) go to the pair two at a time
+    if (f.H % 256 || sms < 2) return MOE_ERR_UNSUPPORTED;
+    return tc_dispatch_pair(f, ws, sms, s);
   }
   return tc_dispatch<KIND_F8, false>(f, ws, sms, s);
 }

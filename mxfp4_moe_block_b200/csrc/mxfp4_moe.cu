@@ -216,7 +216,7 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
   if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
-  if (variant < MOE_FFN_AUTO || variant > MOE_FFN_TENSOR_FUSED) return MOE_ERR_INVALID_ARG;
+  if (variant < MOE_FFN_AUTO || variant > MOE_FFN_TENSOR_F8_PAIR) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !w13_codes || !w13_scales || !w2_codes || !w2_scales || !expert_offsets ||
       !sorted_pair || !y || !workspace)
@@ -240,6 +240,8 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
   if (variant == MOE_FFN_TENSOR_F4) return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F4);
   if (variant == MOE_FFN_TENSOR_FUSED)
     return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F4_FUSED);
+  if (variant == MOE_FFN_TENSOR_F8_PAIR)
+    return tc_ffn(a, ws + wl.tc, dev->sms, s, KIND_F8_PAIR);
   const size_t n8 = (size_t)T * H / 8;
   int st = launched(launch_pdl(x_to_f32_kernel,
                                (unsigned)std::min<size_t>((n8 + 255) / 256, (size_t)dev->sms * 8),

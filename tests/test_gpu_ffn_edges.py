@@ -32,9 +32,10 @@ from gpu_helpers import assert_ffn_close, bf16_to_f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-ALL = [mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED, mm.FFN_AUTO]
+ALL = [mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED,
+       mm.FFN_TENSOR_F8_PAIR, mm.FFN_AUTO]
 NAMES = {mm.FFN_FMA: "fma", mm.FFN_TENSOR_F8: "mxf8f6f4", mm.FFN_TENSOR_F4: "mxf4",
-         mm.FFN_TENSOR_FUSED: "fused", mm.FFN_AUTO: "auto"}
+         mm.FFN_TENSOR_FUSED: "fused", mm.FFN_TENSOR_F8_PAIR: "pair", mm.FFN_AUTO: "auto"}
 
 
 @pytest.fixture(autouse=True)
@@ -118,7 +119,7 @@ def test_format_edge_values_auto_takes_mxf8f6f4():
     sh = synth.Shape("edges", H=1024, I=384, E=16, k=4, S=2, K=8, V=64, seed=2101)
     L = EdgeLayer(sh, empty=(1, 4, 9, 14))
     _edge_values(L)
-    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_AUTO], "edges I=384")
+    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F8_PAIR, mm.FFN_AUTO], "edges I=384")
     with pytest.raises(mm.MoeError) as ei:
         L.run(mm.FFN_TENSOR_F4)
     assert ei.value.status == 2
@@ -184,4 +185,4 @@ def test_scale_matched_blocks_over_the_whole_e8m0_range():
     c = L.w13c[:, :, big]
     lo, hi = c & 0x0F, c >> 4
     L.w13c[:, :, big] = ((lo & 0x0B) | ((hi & 0x0B) << 4)).astype(np.uint8)   # |value| <= 1.5
-    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8], "matched full E8M0")
+    L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F8_PAIR], "matched full E8M0")

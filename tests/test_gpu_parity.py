@@ -178,7 +178,7 @@ def test_ffn_fma(name):
 
 
 @pytest.mark.parametrize("name", ["batch1", "serving", "dflash16", "multilayer"])
-@pytest.mark.parametrize("variant", [3, 4, 5], ids=["mxf8f6f4", "mxf4", "fused"])
+@pytest.mark.parametrize("variant", [3, 4, 5, 6], ids=["mxf8f6f4", "mxf4", "fused", "pair"])
 def test_ffn_tensor(name, variant):
     _ffn_check(name, 0, variant)
 
@@ -186,9 +186,9 @@ def test_ffn_tensor(name, variant):
 def test_ffn_tensor_small_shapes_and_bn_classes():
     """tcgen05 path on small shapes: one expert with many rows (several B
     tiles, a ragged last one), every B-tile width class, and 512+ pairs (the
-    warp-per-row activation encoder, for x and for h); both kinds and the
-    fused launch (in which GEMM-2 tiles wait for their B tile's GEMM-1
-    tiles)."""
+    warp-per-row activation encoder, for x and for h); both kinds, the fused
+    launch (in which GEMM-2 tiles wait for their B tile's GEMM-1 tiles) and
+    the CTA-pair launch (fewer pair tiles than pairs, B halves of 16 rows)."""
     for K, E, k in [(1, 4, 1), (37, 4, 1), (64, 2, 2), (200, 2, 1), (8, 64, 8), (600, 4, 1),
                     (260, 8, 2)]:
         sh = synth.Shape("tcs", H=512, I=256, E=E, k=k, S=1, K=K, V=64, seed=20 + K)
@@ -197,7 +197,8 @@ def test_ffn_tensor_small_shapes_and_bn_classes():
         ridx, _, _ = omoe.route_topk(L.logits_np, sh.k)
         roff, rsp, _ = omoe.permute(ridx, sh.E)
         h_ref, y_ref = omoe.moe_ffn(L.x_f64(), sh.k, sh.I, L.oracle_weights, roff, rsp)
-        for variant in (mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED):
+        for variant in (mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED,
+                        mm.FFN_TENSOR_F8_PAIR):
             y, ws = mm.mxfp4_moe_ffn(L.x, sh.k, *L.w, off, sp, variant=variant)
             assert_ffn_close(bf16_to_f64(mm.workspace_h(ws, sh.P, sh.I)), h_ref,
                              f"h K={K} variant {variant}")

@@ -464,24 +464,6 @@ __device__ __forceinline__ float warp_absmax(float v) {
   return __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(fabsf(v))));
 }
 
-// Two E4M3 terms: codes q[0..1] of this lane, scale bytes sb[0..1] (warp-uniform).
-__device__ __forceinline__ void encode_e4m3x2(float v, uint32_t (&q)[2], uint8_t (&sb)[2]) {
-  float r = v;
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const float amax = warp_absmax(r);
-    int s = 0;
-    uint32_t c = 0;
-    if (amax > 0.f) {
-      s = e4m3_block_exp(amax);
-      c = to_e4m3(r * pow2f(-s));
-      r -= from_e4m3((uint8_t)c) * pow2f(s);
-    }
-    q[t] = c;
-    sb[t] = (uint8_t)(127 + s);
-  }
-}
-
 // Kind of tensor-core MMA used by the FFN (KIND_F4_FUSED: kind::mxf4, both
 // GEMMs in one launch -- a host-side choice only; the kernels see KIND_F4).
 enum TcKind { KIND_F8 = 0, KIND_F4 = 1, KIND_F4_FUSED = 2, KIND_F8_PAIR = 3 };
@@ -517,8 +499,10 @@ __device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two) {
 
 // One whole 32-element block of an activation row, held by one thread: its
 // two E4M3 terms (32 code bytes each, written as two 16-byte stores to q0 and
-// q1) and their scale bytes -- the encoding of encode_e4m3x2, with the block
-// maximum taken over the thread's own values instead of across a warp.
+// q1) and their scale bytes.  Term t takes the scale 2^s with the block's
+// largest remaining magnitude / 2^s in [128, 256) (scale byte 127 + s; an
+// all-zero block gets 127), codes round to nearest, saturating at +-448, and
+// the next term encodes what the codes leave over.
 __device__ __forceinline__ void encode_block_f8(float (&v)[32], uint8_t *q0, uint8_t *q1,
                                                 uint8_t *s0, uint8_t *s1) {
 #pragma unroll
@@ -546,39 +530,44 @@ __device__ __forceinline__ void encode_block_f8(float (&v)[32], uint8_t *q0, uin
   }
 }
 
-// Stores one lane's two E4M3 terms of element n of activation row r (B rows
-// 2r, 2r+1) and, from lane 0, the block's two scale bytes.
-__device__ __forceinline__ void store_terms_f8(float v, size_t r, int n, int kdim,
-                                               uint8_t *q_out, uint8_t *s_out, int lane,
-                                               bool valid) {
-  uint32_t q[2];
-  uint8_t sb[2];
-  encode_e4m3x2(v, q, sb);
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    if (valid) q_out[(2 * r + t) * (size_t)kdim + n] = (uint8_t)q[t];
-    if (valid && lane == 0) s_out[(2 * r + t) * (size_t)(kdim / 32) + n / 32] = sb[t];
-  }
-}
-
 // kind::mxf8f6f4 activation operand of GEMM-1: for every sorted row r (token
 // sp[r]/k) the two E4M3 terms of x[token] as B rows 2r, 2r+1, and their scale
-// bytes.  One warp per 32-element block.
+// bytes.  One thread per 32-element block (four 16-byte loads when x is
+// 16-byte aligned), its maximum taken over its own values: no warp
+// reductions, so the loads of many blocks are in flight at once.
 __global__ void __launch_bounds__(256)
 split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, int P, int k,
                int H, uint8_t *__restrict__ xq, uint8_t *__restrict__ xs, int *counters) {
   pdl_wait();
   pdl_trigger();
   if (counters && blockIdx.x == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
-  const int lane = threadIdx.x & 31;
   const int nb = H / 32;
   const long total = (long)P * nb;
-  for (long w = (blockIdx.x * (long)blockDim.x + threadIdx.x) >> 5; w < total;
-       w += ((long)gridDim.x * blockDim.x) >> 5) {
-    const int r = (int)(w / nb), b = (int)(w % nb);
+  const bool vec = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / nb), b = (int)(i % nb);
     const int t = __ldg(sp + r) / k;
-    const float v = __uint_as_float((uint32_t)__ldg(x + (size_t)t * H + b * 32 + lane) << 16);
-    store_terms_f8(v, (size_t)r, b * 32 + lane, H, xq, xs, lane, true);
+    const uint16_t *src = x + (size_t)t * H + b * 32;
+    float v[32];
+    if (vec) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(src) + q);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * q + 2 * j] = bf16_lo(ww[j]);
+          v[8 * q + 2 * j + 1] = bf16_hi(ww[j]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __uint_as_float((uint32_t)__ldg(src + e) << 16);
+    }
+    const size_t r2 = 2 * (size_t)r;
+    encode_block_f8(v, xq + r2 * H + 32 * b, xq + (r2 + 1) * H + 32 * b, xs + r2 * nb + b,
+                    xs + (r2 + 1) * nb + b);
   }
 }
 
@@ -1962,7 +1951,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       return MOE_ERR_CUDA;
   } else {
     const long blocks = (long)P * (H / 32);
-    const int grid = (int)std::min<long>((blocks * 32 + 255) / 256, (long)sms * 16);
+    const int grid = (int)std::min<long>((blocks + 255) / 256, (long)sms * 16);   // thread per block
     if (launch_pdl(split_x_kernel, grid, 256, 0, s, f.x, f.sp, (int)P, f.k, H, xq, xs, counters) !=
         cudaSuccess)
       return MOE_ERR_CUDA;

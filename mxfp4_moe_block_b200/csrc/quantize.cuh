@@ -59,8 +59,8 @@ __device__ __forceinline__ uint32_t quantize_group8(const uint4 v, uint32_t *sb)
 // w: n8 groups of 8 bf16 (n8 = R*K/8); codes: 4 bytes per group; scales: one
 // byte per 4 groups.  Each warp takes QUANT_UNROLL runs of 32 consecutive
 // groups per trip, all loads first, so that each thread keeps QUANT_UNROLL
-// 16-byte loads in flight.
-constexpr int QUANT_UNROLL = 4;
+// 16-byte loads in flight (8: 0.92 of the copy bandwidth, against 0.77 with 4).
+constexpr int QUANT_UNROLL = 8;
 
 __global__ void __launch_bounds__(QUANT_THREADS)
 mxfp4_quantize_kernel(const uint16_t *__restrict__ w, size_t n8, uint8_t *__restrict__ codes,

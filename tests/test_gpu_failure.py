@@ -4,7 +4,9 @@ The tensor-core FFN bounds every wait it makes.  Here the limit is lowered
 far below a kernel's run time (moe_set_wait_limit_ns), so a wait runs out:
 the kernel must report MOE_DEV_TIMEOUT through the device status word, drain
 the copies and MMAs it issued, free its tensor memory and return, leaving the
-context usable -- the next call, at the normal limit, matches the oracle.
+context usable -- the next call, at the normal limit, matches the oracle.  The
+CTA-pair launch also tells the partner CTA, which holds operands and barriers
+of the same MMAs, and the two leave together.
 
 The library's per-device set-up (kernel attributes, the tensor-map encoder)
 must also survive two host threads making their first calls at once.
@@ -40,8 +42,9 @@ def _problem():
     return sh, L, off, sp, h_ref, y_ref
 
 
-@pytest.mark.parametrize("variant", [mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED],
-                         ids=["mxf8f6f4", "mxf4", "fused"])
+@pytest.mark.parametrize("variant", [mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F4, mm.FFN_TENSOR_FUSED,
+                                     mm.FFN_TENSOR_F8_PAIR],
+                         ids=["mxf8f6f4", "mxf4", "fused", "pair"])
 def test_wait_timeout_reports_and_context_recovers(variant):
     sh, L, off, sp, h_ref, y_ref = _problem()
     timed_out = False

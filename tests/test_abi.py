@@ -54,3 +54,28 @@ def test_host_only_calls(library):
     # a vocabulary beyond the greedy key's 26 token bits is refused up front
     # (non-null dummy addresses: the size check comes before any device use)
     assert library.block_accept_greedy(16, 16, 1, 8, (1 << 26) + 1, 16, 16, None) == 2
+
+
+def header_enum_values(prefix):
+    """Name -> value of the header's enumerators that start with `prefix`."""
+    vals = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h, encoding="utf-8").read(), flags=re.S)
+        for m in re.finditer(r"\b(" + prefix + r"\w*)\s*=\s*(-?\d+)", text):
+            vals[m.group(1)] = int(m.group(2))
+    return vals
+
+
+def test_ffn_variant_constants_match_the_header():
+    v = header_enum_values("MOE_FFN_")
+    assert v == {"MOE_FFN_AUTO": 0, "MOE_FFN_FMA": 1, "MOE_FFN_TENSOR": 2, "MOE_FFN_TENSOR_F8": 3,
+                 "MOE_FFN_TENSOR_F4": 4, "MOE_FFN_TENSOR_FUSED": 5, "MOE_FFN_TENSOR_F8_PAIR": 6}
+    for name, val in v.items():
+        assert getattr(_lib, name[len("MOE_"):]) == val, name
+
+
+def test_variant_range_is_checked(library):
+    # a variant past the last enumerator is refused before any device use
+    last = max(header_enum_values("MOE_FFN_").values())
+    assert library.mxfp4_moe_ffn_variant(None, 1, 512, 256, 8, 2, None, None, None, None,
+                                         None, None, None, None, 0, last + 1, None) == 1

@@ -53,7 +53,9 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="batch1", choices=list(synth.SHAPES))
-    ap.add_argument("--variant", type=int, default=0, help="FFN kernel: 0 auto, 1 FMA, 2 tensor")
+    ap.add_argument("--variant", type=int, default=0,
+                    help="FFN kernel: 0 auto, 1 FMA, 2 tensor, 3 kind::mxf8f6f4, 4 kind::mxf4, "
+                         "5 fused, 6 kind::mxf8f6f4 on CTA pairs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
@@ -110,6 +112,9 @@ def _profile_value(fname, key):
         return float(kv[key])
     except Exception:
         return None
+
+
+VARIANT_NAMES = {0: "auto", 1: "fma", 2: "tensor", 3: "mxf8f6f4", 4: "mxf4", 5: "fused", 6: "pair"}
 
 
 def load_traffic(workload, variant_name):
@@ -697,7 +702,7 @@ def measure_config(name, variant, steps, warmup, device, peaks, clocks, with_cpu
     t = time_steps(wl, variant, steps, warmup, True, clocks)
     n_launch, _ = count_launches(wl, variant)
     acc = wl.accepted()
-    vname = {0: "auto", 1: "fma", 2: "tensor"}.get(variant, str(variant))
+    vname = VARIANT_NAMES.get(variant, str(variant))
     entry = {
         "config": workload_config(sh, 1),
         "ms_per_step": t["ms"], "timing": t["timing"],
@@ -771,7 +776,7 @@ def main():
     mm.lib()
     peaks = load_peaks()
     variant = args.variant
-    vname = {0: "auto", 1: "fma", 2: "tensor"}.get(variant, str(variant))
+    vname = VARIANT_NAMES.get(variant, str(variant))
 
     def barrier():
         if world > 1:

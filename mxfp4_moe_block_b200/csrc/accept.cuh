@@ -165,7 +165,6 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
   __shared__ int s_a;
   __shared__ unsigned long long s_red[32];
-  __shared__ int s_found;
 
   if (w == 0) {
     bool acc = true;
@@ -182,10 +181,7 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
       }
     }
     const unsigned rej = __ballot_sync(FULL, lane < K && !acc);
-    if (lane == 0) {
-      s_a = rej ? __ffs(rej) - 1 : K;
-      s_found = 0;
-    }
+    if (lane == 0) s_a = rej ? __ffs(rej) - 1 : K;
   }
   __syncthreads();
   const int a = s_a;
@@ -202,11 +198,15 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
   const unsigned long long U = (unsigned long long)((double)__ldg(u_resample + s) * 16777216.0);
 
   // weight of token v: floor(max(0, p-q) * 2^40), or floor(p * 2^40) (mode 1)
-  auto weight = [&](int v, int mode) -> unsigned long long {
-    const float pv = __ldg(pr + v);
-    const float r = mode ? pv : fmaxf(__fsub_rn(pv, __ldg(qr + v)), 0.f);
+  auto weight_of = [](float pv, float qv, int mode) -> unsigned long long {
+    const float r = mode ? pv : fmaxf(__fsub_rn(pv, qv), 0.f);
     return (unsigned long long)((double)r * 1099511627776.0);
   };
+  auto weight = [&](int v, int mode) -> unsigned long long {
+    return weight_of(__ldg(pr + v), mode ? 0.f : __ldg(qr + v), mode);
+  };
+  // rows of whole 16-byte groups (the chunk below is then a multiple of 128)
+  const bool vec4 = (V & 3) == 0 && ((reinterpret_cast<uintptr_t>(pr) | reinterpret_cast<uintptr_t>(qr)) & 15) == 0;
   auto block_sum = [&](unsigned long long x) -> unsigned long long {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
@@ -218,48 +218,88 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
     return t;
   };
 
-  const int tile = blockDim.x;   // one element per thread per tile, coalesced
+  // Warp w owns the contiguous range [w*chunk, (w+1)*chunk) of the row: its
+  // lanes sum the weights there (consecutive lanes, consecutive tokens), the
+  // block adds the warp sums, and only the warp whose range holds the target
+  // mass scans it.  The weights are integers, so every order of adding them
+  // gives the same sums and the same token.
+  const int chunk = (((V + nw - 1) / nw) + 127) & ~127;
+  const int c0 = min(V, w * chunk), c1 = min(V, c0 + chunk);
   // the bonus draw takes p itself (mode 1) at once
   for (int mode = a == K ? 1 : 0; mode < 2; ++mode) {
     unsigned long long mine = 0;
-    for (int v = tid; v < V; v += tile) mine += weight(v, mode);
-    const unsigned long long total = block_sum(mine);
+    if (vec4) {
+      // 16-byte loads: lane l takes tokens c0 + 4(l + 32i) .. +3 (chunk is a
+      // multiple of 128 here, so every group of four lies in one warp's range)
+      for (int v = c0 + 4 * lane; v < c1; v += 4 * 128) {
+        float4 pv[4], qv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int vj = v + 128 * j;
+          pv[j] = vj < c1 ? __ldg(reinterpret_cast<const float4 *>(pr + vj)) : make_float4(0, 0, 0, 0);
+          qv[j] = (vj < c1 && !mode) ? __ldg(reinterpret_cast<const float4 *>(qr + vj))
+                                     : make_float4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          mine += weight_of(pv[j].x, qv[j].x, mode) + weight_of(pv[j].y, qv[j].y, mode) +
+                  weight_of(pv[j].z, qv[j].z, mode) + weight_of(pv[j].w, qv[j].w, mode);
+        }
+      }
+    } else {
+      for (int v = c0 + lane; v < c1; v += 4 * 32) {
+        unsigned long long x[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[j] = v + 32 * j < c1 ? weight(v + 32 * j, mode) : 0ull;
+        mine += (x[0] + x[1]) + (x[2] + x[3]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(FULL, mine, o);
+    __syncthreads();                         // s_red is free (a previous mode read it)
+    if (lane == 0) s_red[w] = mine;
+    __syncthreads();
+    unsigned long long total = 0;
+    for (int j = 0; j < nw; ++j) total += s_red[j];
     if (total == 0) continue;
     // target mass m = floor(total * U / 2^24), total < 2^58, U < 2^24
     const unsigned long long lo = total * U, hi = __umul64hi(total, U);
     const unsigned long long m = (hi << 40) | (lo >> 24);
-    unsigned long long run = 0;   // mass of all tiles before this one
-    for (int base = 0; base < V; base += tile) {
-      const int v = base + tid;
-      const unsigned long long wv = v < V ? weight(v, mode) : 0ull;
-      // inclusive scan of wv over the block
-      unsigned long long x = wv;
+    // the warp whose range holds mass m: its prefix is <= m < prefix + sum
+    unsigned long long before = 0;
+    for (int j = 0; j < w; ++j) before += s_red[j];
+    // every other warp is done (no barrier follows: the owner scans alone)
+    if (!(before <= m && m < before + s_red[w])) return;
+    unsigned long long run = before;
+    for (int b0 = c0; b0 < c1; b0 += 4 * 32) {
+      unsigned long long wq[4];              // four steps' weights, loaded together
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long y = __shfl_up_sync(FULL, x, o);
-        if (lane >= o) x += y;
+      for (int j = 0; j < 4; ++j) {
+        const int v = b0 + 32 * j + lane;
+        wq[j] = v < c1 ? weight(v, mode) : 0ull;
       }
-      __syncthreads();
-      if (lane == 31) s_red[w] = x;
-      __syncthreads();
-      unsigned long long before_w = 0, tile_sum = 0;
-      for (int j = 0; j < nw; ++j) {
-        if (j < w) before_w += s_red[j];
-        tile_sum += s_red[j];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = b0 + 32 * j + lane;
+        const unsigned long long wv = wq[j];
+        unsigned long long x = wv;           // inclusive scan over the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long y = __shfl_up_sync(FULL, x, o);
+          if (lane >= o) x += y;
+        }
+        const unsigned long long incl = run + x;
+        // the token: the first v whose inclusive prefix exceeds m
+        const bool hit = wv > 0 && incl > m && incl - wv <= m;
+        if (hit) next_token[s] = v;
+        if (__any_sync(FULL, hit)) return;
+        run += __shfl_sync(FULL, x, 31);
       }
-      const unsigned long long incl = run + before_w + x;
-      // the token: first v whose inclusive prefix exceeds m
-      if (wv > 0 && incl > m && incl - wv <= m) {
-        next_token[s] = v;
-        s_found = 1;
-      }
-      __syncthreads();
-      if (s_found) return;
-      run += tile_sum;
     }
-    raise_status(MOE_DEV_NO_MASS);   // not reached: m < total always finds a token
+    if (lane == 0) raise_status(MOE_DEV_NO_MASS);   // not reached: the warp holds mass m
     return;
   }
+  // no mode had any mass (total is the same in every thread, so all reach here)
   if (tid == 0) {
     raise_status(MOE_DEV_NO_MASS);
     next_token[s] = -1;

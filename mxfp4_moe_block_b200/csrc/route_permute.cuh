@@ -76,6 +76,8 @@ route_topk_kernel(const float *__restrict__ logits, int T, int E, int k,
 // Dynamic shared memory: 32*E counters + E offsets (ints).
 // topk_idx is read with plain loads: the fused kernel below writes it in
 // the same launch.
+constexpr int PERM_BATCH = 8;   // steps of 32 pairs whose ids a lane loads at once
+
 __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, int E,
                                               int32_t *__restrict__ expert_offsets,
                                               int32_t *__restrict__ sorted_pair,
@@ -90,23 +92,31 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
 
   for (int e = lane; e < E; e += 32) cnt[w * E + e] = 0;
   __syncwarp();
-  // pass A
-  for (int base = p0; base < p1; base += 32) {
-    const int p = base + lane;
-    int e = -1;
-    if (p < p1) {
-      e = topk_idx[p];
-      if (e < 0 || e >= E) { raise_status(MOE_DEV_BAD_EXPERT); e = -1; }
+  // pass A.  The lane's expert ids for PERM_BATCH steps of 32 pairs are
+  // loaded first (independent loads in flight), then ranked step by step.
+  for (int b0 = p0; b0 < p1; b0 += 32 * PERM_BATCH) {
+    int ev[PERM_BATCH];
+#pragma unroll
+    for (int j = 0; j < PERM_BATCH; ++j) {
+      const int p = b0 + 32 * j + lane;
+      ev[j] = p < p1 ? topk_idx[p] : -1;
     }
-    const unsigned same = __match_any_sync(FULL, e);
-    int before = 0;
-    if (e >= 0) before = cnt[w * E + e];
-    __syncwarp();
-    if (e >= 0) {
-      pair_row[p] = before + __popc(same & lanemask_lt());
-      if ((same & lanemask_lt()) == 0) cnt[w * E + e] = before + __popc(same);
+#pragma unroll
+    for (int j = 0; j < PERM_BATCH; ++j) {
+      const int p = b0 + 32 * j + lane;
+      int e = ev[j];
+      if (p < p1 && (e < 0 || e >= E)) { raise_status(MOE_DEV_BAD_EXPERT); e = -1; }
+      if (p >= p1) e = -1;
+      const unsigned same = __match_any_sync(FULL, e);
+      int before = 0;
+      if (e >= 0) before = cnt[w * E + e];
+      __syncwarp();
+      if (e >= 0) {
+        pair_row[p] = before + __popc(same & lanemask_lt());
+        if ((same & lanemask_lt()) == 0) cnt[w * E + e] = before + __popc(same);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   }
   __syncthreads();
   // pass B: per expert, exclusive prefix over warps (E <= 1024, checked on
@@ -145,13 +155,21 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
     if (e == E - 1) expert_offsets[E] = incl;
   }
   __syncthreads();
-  // pass C
-  for (int base = p0; base < p1; base += 32) {
-    const int p = base + lane;
-    if (p < p1) {
-      const int e = topk_idx[p];
-      if (e >= 0 && e < E) {
-        const int pos = offs[e] + cnt[w * E + e] + pair_row[p];
+  // pass C (the same batching)
+  for (int b0 = p0; b0 < p1; b0 += 32 * PERM_BATCH) {
+    int ev[PERM_BATCH], rk[PERM_BATCH];
+#pragma unroll
+    for (int j = 0; j < PERM_BATCH; ++j) {
+      const int p = b0 + 32 * j + lane;
+      ev[j] = p < p1 ? topk_idx[p] : -1;
+      rk[j] = p < p1 ? pair_row[p] : 0;
+    }
+#pragma unroll
+    for (int j = 0; j < PERM_BATCH; ++j) {
+      const int p = b0 + 32 * j + lane;
+      const int e = ev[j];
+      if (p < p1 && e >= 0 && e < E) {
+        const int pos = offs[e] + cnt[w * E + e] + rk[j];
         sorted_pair[pos] = p;
         pair_row[p] = pos;
       }

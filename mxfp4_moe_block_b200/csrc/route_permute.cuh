@@ -107,7 +107,15 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
       int e = ev[j];
       if (p < p1 && (e < 0 || e >= E)) { raise_status(MOE_DEV_BAD_EXPERT); e = -1; }
       if (p >= p1) e = -1;
-      const unsigned same = __match_any_sync(FULL, e);
+      // lanes holding the same expert: the bits of e (-1 taken as 1024, E <=
+      // 1024) by ballots -- 11 ballots cost less than __match_any_sync here
+      const unsigned key = e < 0 ? 1024u : (unsigned)e;
+      unsigned same = FULL;
+#pragma unroll
+      for (int bit = 0; bit < 11; ++bit) {
+        const unsigned bb = __ballot_sync(FULL, (key >> bit) & 1u);
+        same &= ((key >> bit) & 1u) ? bb : ~bb;
+      }
       int before = 0;
       if (e >= 0) before = cnt[w * E + e];
       __syncwarp();

@@ -207,16 +207,6 @@ rejection_kernel(const float *__restrict__ p, const float *__restrict__ q,
   };
   // rows of whole 16-byte groups (the chunk below is then a multiple of 128)
   const bool vec4 = (V & 3) == 0 && ((reinterpret_cast<uintptr_t>(pr) | reinterpret_cast<uintptr_t>(qr)) & 15) == 0;
-  auto block_sum = [&](unsigned long long x) -> unsigned long long {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
-    __syncthreads();
-    if (lane == 0) s_red[w] = x;
-    __syncthreads();
-    unsigned long long t = 0;
-    for (int j = 0; j < nw; ++j) t += s_red[j];
-    return t;
-  };
 
   // Warp w owns the contiguous range [w*chunk, (w+1)*chunk) of the row: its
   // lanes sum the weights there (consecutive lanes, consecutive tokens), the

@@ -763,6 +763,10 @@ inline cudaError_t launch_encode_f4(const uint16_t *src, const int32_t *sp, int 
 struct TcMaps {
   CUtensorMap a;        // weights [E*rows, K]: box 128 (padded E2M1) or 128 B (packed) x 64 rows
   CUtensorMap b[4];     // activation terms [T*P, row bytes]: box 128 B x {16, 32, 64, 128} rows
+  // scale bytes in 16-byte groups (TcArgs::sf_tma): weights [E*rows, K/32],
+  // box 16 B x 64 rows; activation terms [T*P, K/32], box 16 B x the B boxes' rows
+  CUtensorMap sa;
+  CUtensorMap sb[4];
 };
 
 struct TcArgs {
@@ -787,6 +791,9 @@ struct TcArgs {
   // readiness flag (zeroed by the same encode kernel)
   int *bt_done;
   int *bt_ready;
+  // kind::mxf8f6f4, K % 512 == 0 (16 scale bytes per row cover four
+  // stages): the scale bytes come by TMA through maps sa / sb
+  int sf_tma;
 };
 
 constexpr int kMaxStages = 12;
@@ -808,10 +815,21 @@ struct TcCfg {
   // ahead; sized to leave the operand stages as many as before.  Else one
   // scale slot per operand stage.
   static constexpr int kSfRing = KIND == KIND_F8 ? (PAIR ? 8 : 4) : 0;
+  // With TcArgs::sf_tma the scale bytes come instead in groups of kSfGroup
+  // stages (16 bytes of each A and B row) by TMA, into one of kSftSlots
+  // slots of [128 A rows][16] then [BN B rows][16] bytes.
+  static constexpr int kSfGroup = 16 / (4 * Kd::kKGroups);
+  static constexpr int kSftA = 128 * 16;               // A part of a slot; the B part follows
+  static constexpr int kSft = KIND == KIND_F8 ? kSftA + 16 * BN : 0;   // all B rows (PAIR too)
+  static constexpr int kSftSlots = 2;
+  static constexpr int kRingBytes =
+      !kSfRing ? 0
+               : (kSfRing * (kSfa + kSfb) > kSftSlots * kSft ? kSfRing * (kSfa + kSfb)
+                                                              : kSftSlots * kSft);
   static constexpr int kStageBytes = kA + kB + (kSfRing ? 0 : kSfa + kSfb);
   static constexpr int kFixed = 1024 + Kd::kEpiGroups * 64 * (16 / Kd::kTerms) * 4 + 1026 * 2 +
                                  2 * 1025 * 4 + 128 + 1024 + kSfbConst;
-  static constexpr int kStages0 = (227 * 1024 - kFixed - kSfRing * (kSfa + kSfb)) / kStageBytes;
+  static constexpr int kStages0 = (227 * 1024 - kFixed - kRingBytes) / kStageBytes;
   static constexpr int kStages = kStages0 > kMaxStages ? kMaxStages : kStages0;
   static constexpr int kSfSlots = kSfRing ? kSfRing : kStages;
   static constexpr int kSfCols =                                    // TMEM columns per stage
@@ -832,7 +850,7 @@ struct TcCfg {
   static constexpr int kOffB = kStages * kA;
   static constexpr int kOffSfa = kOffB + kStages * kB;
   static constexpr int kOffSfb = kOffSfa + kSfSlots * kSfa;
-  static constexpr int kOffBar = kOffSfb + kSfSlots * kSfb;
+  static constexpr int kOffBar = kSfRing ? kOffSfa + kRingBytes : kOffSfb + kSfSlots * kSfb;
   // SwiGLU exchange: 64 rows x (tokens per 16-column chunk) floats per
   // epilogue warp group
   static constexpr int kXchgFloats = 64 * (16 / Kd::kTerms);
@@ -843,9 +861,18 @@ struct TcCfg {
   static constexpr int kOffSfbConst = (kOffTab + kTabBytes + 127) & ~127;  // 16B-aligned for tcgen05.cp
   static constexpr int kSmem = kOffSfbConst + kSfbConst + 1024;   // + alignment slack
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
-  static_assert(kOffSfa % 1024 == 0 && kOffSfb % 128 == 0 && kOffSfbConst % 128 == 0,
-                "descriptor alignment");
+  static_assert(kOffSfa % 1024 == 0 && kOffSfb % 128 == 0 && kOffSfbConst % 128 == 0 &&
+                    kSft % 128 == 0,
+                "descriptor and TMA destination alignment");
 };
+
+// B rows of a tile (N = ncol, a multiple of 16): one box of 16, 32, 64 or
+// 128 rows, or a 128-row box and a second one for the rest.  Box class
+// (0..3) | (class of the second box + 1) << 3.
+__device__ __forceinline__ int b_box_class(int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; }
+__device__ __forceinline__ int b_box_sel(int ncol) {
+  return ncol <= 128 ? b_box_class(ncol) : 3 | ((b_box_class(ncol - 128) + 1) << 3);
+}
 
 // warps: 0 TMA producer, 1 scale loader, 2 TMEM + MMA issuer, 3 constant B
 // scales, 4-7 epilogue, 8-11 scale writers (one per TMEM lane quarter),
@@ -941,6 +968,9 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   // the table's prefix is in tiles (MODES 1, 2; PAIR: tiles of two
   // m-blocks) or in B tiles (MODE 3)
   const int mtiles = MODE == 3 ? 1 : PAIR ? mt1 / 2 : mt1;
+  // scale bytes by TMA in 16-byte groups (kind::mxf8f6f4)
+  const bool sft = KIND == KIND_F8 && MODE != 3 && a.sf_tma != 0;
+  const int n_sfslots = sft ? C::kSftSlots : C::kSfSlots;
 
   // tile table: active experts and the prefix of their tile counts
   if (warp == 0) {
@@ -981,7 +1011,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       if (PAIR) mbar_init(&ready[s], 8);
     }
     for (int s = 0; s < C::kSfSlots; ++s) {
-      mbar_init(&sfs_full[s], 32);     // 32 scale-loader lanes (cp.async)
+      mbar_init(&sfs_full[s], sft ? 1 : 32);   // the loader's expect_tx, or 32 cp.async lanes
       if (C::kSfRing) mbar_init(&sfs_empty[s], 4);   // 4 scale-writer warps
     }
     for (int r = 0; r < kRing; ++r) {
@@ -1073,22 +1103,18 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      // B rows of a tile: one box of 16, 32, 64 or 128 rows, or -- wider
-      // tiles -- a 128-row box and a second one for the rest, so a stage
-      // loads at most 15 rows more than the tile's N.  bsel = box class
-      // (0..3) | (class of the second box + 1) << 3.
-      auto box_class = [](int n) { return n <= 16 ? 0 : n <= 32 ? 1 : n <= 64 ? 2 : 3; };
-      // PAIR: N rounded up to 32, this CTA's half (a multiple of 16 rows)
-      // in one box of up to 64 rows or a 64-row box and a second one.
+      // B rows of a tile: b_box_sel's boxes, so a stage loads at most 15
+      // rows more than the tile's N.  PAIR: N rounded up to 32, this CTA's
+      // half (a multiple of 16 rows) in one box of up to 64 rows or a 64-row
+      // box and a second one.
       auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel, int &ph, int &g) {
         const Tile tl = decode(t);
         if (PAIR) {
           const int half = ((tl.nB + 31) & ~31) / 2;
-          bsel = half <= 64 ? box_class(half) : 2 | ((box_class(half - 64) + 1) << 3);
+          bsel = half <= 64 ? b_box_class(half) : 2 | ((b_box_class(half - 64) + 1) << 3);
           rowB = tl.rowB + (int)crank * half;
         } else {
-          const int ncol = (tl.nB + 15) & ~15;
-          bsel = ncol <= 128 ? box_class(ncol) : 3 | ((box_class(ncol - 128) + 1) << 3);
+          bsel = b_box_sel((tl.nB + 15) & ~15);
           rowB = tl.rowB;
         }
         ph = tl.ph;
@@ -1191,64 +1217,108 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     }
   } else if (warp == 1) {
     // --------------------------------------------------- scale loader --
-    // Per stage and 4-scale group g: scale bytes of the 128 A rows (and of
-    // the B rows) go straight into the 32 x 16-byte layout of tcgen05.cp:
-    // byte 16*(row%32) + 4*(row/32) + (k-block within the group).
+    // cp.async path: per stage and 4-scale group g, the scale bytes of the
+    // 128 A rows (and of the B rows) go straight into the 32 x 16-byte layout
+    // of the scale-factor columns: byte 16*(row%32) + 4*(row/32) + (k-block
+    // within the group).
     if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
-    // Leave-or-stay decisions are warp-wide, so that every stage this warp
-    // signals gets all 32 lanes' arrivals.
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int ti = 0; ok; ++ti) {
-      const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
-      if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
-      const Tile tl = decode(t);
-      const int mt = tl.mt, rowB = tl.rowB, nB = tl.nB;
-      const TcArgs &ap = tl.ph ? a2 : a;       // this phase's operands
-      const uint32_t kb = ap.K / 32;           // scale bytes per row
-      const int ebase = tl.e * ap.rows_per_expert;
-      // this lane's four A rows (lane + 32q) for the whole tile
-      const uint8_t *src_a[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i = lane + 32 * q;
-        const int row = mode_of(tl.ph) == 1
-                            ? ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64)
-                            : ebase + mt * 128 + i;
-        src_a[q] = ap.a_scales + (size_t)row * kb;
-      }
-      const int ksteps = ksteps_of(tl.ph);
-      for (int kt = 0; kt < ksteps; ++kt) {
-        // the slot is free: its last bytes are in tensor memory (kSfRing), or
-        // the MMAs that read its stage's columns are done
-        if (!__all_sync(FULL, C::kSfRing ? mbar_wait_fast(&sfs_empty[stage], phase ^ 1, abort)
-                                         : mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
-          ok = false;
-          break;
-        }
-        uint8_t *sfa = smem + C::kOffSfa + stage * C::kSfa;
-        uint8_t *sfb = smem + C::kOffSfb + stage * C::kSfb;
-#pragma unroll
-        for (int g = 0; g < Kd::kKGroups; ++g) {
-          const uint32_t koff = (uint32_t)(kt * Kd::kKGroups + g) * 4;
-#pragma unroll
-          for (int q = 0; q < 4; ++q)         // A rows lane + 32q
-            cp_async4(sfa + 512 * g + 16 * lane + 4 * q, src_a[q] + koff);
-#pragma unroll
-          for (int q = 0; q < 4 * C::kRowChunks; ++q) {
-            const int i = lane + 32 * q;
-            if (!Kd::kRowScaledB && i < nB)
-              cp_async4(sfb + 512 * (g * C::kRowChunks + (q >> 2)) + 16 * lane + 4 * (q & 3),
-                        ap.b_scales + (size_t)(rowB + i) * kb + koff);
+    if (sft) {
+      // 16 bytes of every A row and B row of the tile -- the scale bytes of
+      // kSfGroup stages -- per TMA group: the two 64-row halves of the weight
+      // tile, then the B tile's boxes (evict-first and evict-last, as their
+      // operands), into a slot of [row][16] bytes.  The writer warps free a
+      // slot as soon as they have read it, at the group's first stage.
+      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      int slot = 0;
+      uint32_t sph = 0;
+      bool ok = true;
+      for (int ti = 0; ok; ++ti) {
+        const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+        if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
+        const Tile tl = decode(t);
+        const int arow = tl.e * a.rows_per_expert + (MODE == 1 ? tl.mt * 64 : tl.mt * 128);
+        const int arow2 = arow + (MODE == 1 ? a.I : 64);
+        const int bsel = b_box_sel((tl.nB + 15) & ~15);
+        const int tail = bsel >> 3;
+        const uint32_t bytes =
+            (uint32_t)(C::kSftA + 16 * (a.b_box[bsel & 7] + (tail ? a.b_box[tail - 1] : 0)));
+        const int groups = ksteps_of(tl.ph) / C::kSfGroup;
+        for (int gi = 0; gi < groups; ++gi) {
+          if (!__all_sync(FULL, mbar_wait_fast(&sfs_empty[slot], sph ^ 1, abort))) {
+            ok = false;
+            break;
           }
+          if (lane == 0) {
+            uint8_t *dst = smem + C::kOffSfa + slot * C::kSft;
+            mbar_expect_tx(&sfs_full[slot], bytes);
+            tma_load_2d(dst, &maps.sa, 16 * gi, arow, &sfs_full[slot], pol_w);
+            tma_load_2d(dst + 64 * 16, &maps.sa, 16 * gi, arow2, &sfs_full[slot], pol_w);
+            tma_load_2d(dst + C::kSftA, &maps.sb[bsel & 7], 16 * gi, tl.rowB, &sfs_full[slot],
+                        pol_x);
+            if (tail)
+              tma_load_2d(dst + C::kSftA + 128 * 16, &maps.sb[tail - 1], 16 * gi, tl.rowB + 128,
+                          &sfs_full[slot], pol_x);
+          }
+          ++l_signaled;
+          if (++slot == C::kSftSlots) { slot = 0; sph ^= 1; }
         }
-        cp_async_arrive_noinc(&sfs_full[stage]);
-        ++l_signaled;
-        if (++stage == C::kSfSlots) { stage = 0; phase ^= 1; }
       }
+    } else {
+      // Leave-or-stay decisions are warp-wide, so that every stage this warp
+      // signals gets all 32 lanes' arrivals.
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int ti = 0; ok; ++ti) {
+        const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
+        if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
+        const Tile tl = decode(t);
+        const int mt = tl.mt, rowB = tl.rowB, nB = tl.nB;
+        const TcArgs &ap = tl.ph ? a2 : a;       // this phase's operands
+        const uint32_t kb = ap.K / 32;           // scale bytes per row
+        const int ebase = tl.e * ap.rows_per_expert;
+        // this lane's four A rows (lane + 32q) for the whole tile
+        const uint8_t *src_a[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i = lane + 32 * q;
+          const int row = mode_of(tl.ph) == 1
+                              ? ebase + (i < 64 ? mt * 64 + i : a.I + mt * 64 + i - 64)
+                              : ebase + mt * 128 + i;
+          src_a[q] = ap.a_scales + (size_t)row * kb;
+        }
+        const int ksteps = ksteps_of(tl.ph);
+        for (int kt = 0; kt < ksteps; ++kt) {
+          // the slot is free: its last bytes are in tensor memory (kSfRing), or
+          // the MMAs that read its stage's columns are done
+          if (!__all_sync(FULL, C::kSfRing ? mbar_wait_fast(&sfs_empty[stage], phase ^ 1, abort)
+                                           : mbar_wait_fast(&empty[stage], phase ^ 1, abort))) {
+            ok = false;
+            break;
+          }
+          uint8_t *sfa = smem + C::kOffSfa + stage * C::kSfa;
+          uint8_t *sfb = smem + C::kOffSfb + stage * C::kSfb;
+#pragma unroll
+          for (int g = 0; g < Kd::kKGroups; ++g) {
+            const uint32_t koff = (uint32_t)(kt * Kd::kKGroups + g) * 4;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)         // A rows lane + 32q
+              cp_async4(sfa + 512 * g + 16 * lane + 4 * q, src_a[q] + koff);
+#pragma unroll
+            for (int q = 0; q < 4 * C::kRowChunks; ++q) {
+              const int i = lane + 32 * q;
+              if (!Kd::kRowScaledB && i < nB)
+                cp_async4(sfb + 512 * (g * C::kRowChunks + (q >> 2)) + 16 * lane + 4 * (q & 3),
+                          ap.b_scales + (size_t)(rowB + i) * kb + koff);
+            }
+          }
+          cp_async_arrive_noinc(&sfs_full[stage]);
+          ++l_signaled;
+          if (++stage == C::kSfSlots) { stage = 0; phase ^= 1; }
+        }
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 2) {
     // ----------------------------------------------------- MMA issuer --
     if (PAIR && !leader && lane == 0) {
@@ -1366,6 +1436,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     uint32_t phase = 0;
     int slot = 0;          // scale slot (the stage itself unless kSfRing)
     uint32_t sph = 0;
+    int sub = 0;           // sft: the stage's place in its group
+    // sft: the group's 16 bytes of this lane's A rows (32j + lane) and B rows
+    // (128c + 32j + lane), taken out of the slot at the group's first stage
+    // so that the loader can refill it at once; .x is the current stage's
+    uint4 ga[4], gb[C::kRowChunks][4];
     bool ok = true;
     for (int ti = 0; ok; ++ti) {
       const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
@@ -1375,37 +1450,77 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         // the MMAs that read this stage's columns last time are done, and the
         // stage's scale bytes are in shared memory
         const bool rdy = mbar_wait_fast(&empty[stage], phase ^ 1, abort) &&
-                         mbar_wait_fast(&sfs_full[slot], sph, abort);
+                         ((sft && sub != 0) || mbar_wait_fast(&sfs_full[slot], sph, abort));
         if (!__all_sync(FULL, rdy)) { ok = false; break; }
         tc_fence_after();
-        const uint4 *src =
-            reinterpret_cast<const uint4 *>(smem + C::kOffSfa + slot * C::kSfa) + lane;
         const uint32_t dst = tmem + lane_base + (uint32_t)C::kAccCols + stage * C::kSfCols;
-        if (Kd::kKGroups == 2) {
-          const uint4 g0 = src[0], g1 = src[32];
-          const uint32_t r[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-          tc_st_x8(dst, r);
-        } else {
-          const uint4 g0 = src[0];
-          const uint32_t r[4] = {g0.x, g0.y, g0.z, g0.w};
-          tc_st_x4(dst, r);
-        }
-        if (!Kd::kRowScaledB) {
-          // kind::mxf8f6f4's B block scales: the same layout, one 128-row
-          // chunk of B after another, behind the A scale columns
-          const uint4 *srb =
-              reinterpret_cast<const uint4 *>(smem + C::kOffSfb + slot * C::kSfb) + lane;
+        if (sft) {
+          if (sub == 0) {
+            // [row][16] bytes; B rows past the tile's boxes feed no output
+            // column
+            const uint4 *sv = reinterpret_cast<const uint4 *>(smem + C::kOffSfa + slot * C::kSft);
 #pragma unroll
-          for (int gc = 0; gc < Kd::kKGroups * C::kRowChunks; ++gc) {
-            const uint4 v = srb[32 * gc];
-            const uint32_t r[4] = {v.x, v.y, v.z, v.w};
-            tc_st_x4(dst + 4 * Kd::kKGroups + 4 * gc, r);
+            for (int j = 0; j < 4; ++j) ga[j] = sv[32 * j + lane];
+#pragma unroll
+            for (int c = 0; c < C::kRowChunks; ++c)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int row = 128 * c + 32 * j + lane;
+                gb[c][j] = row < BN ? sv[C::kSftA / 16 + row] : make_uint4(0u, 0u, 0u, 0u);
+              }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfs_empty[slot]);   // after the warp's reads
+            if (++slot == C::kSftSlots) { slot = 0; sph ^= 1; }
+          }
+          uint32_t r[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) r[j] = ga[j].x;
+          tc_st_x4(dst, r);
+#pragma unroll
+          for (int c = 0; c < C::kRowChunks; ++c) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) r[j] = gb[c][j].x;
+            tc_st_x4(dst + 4 + 4 * c, r);
+          }
+          // the next stage's bytes move into .x
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ga[j] = make_uint4(ga[j].y, ga[j].z, ga[j].w, 0u);
+#pragma unroll
+          for (int c = 0; c < C::kRowChunks; ++c)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              gb[c][j] = make_uint4(gb[c][j].y, gb[c][j].z, gb[c][j].w, 0u);
+        } else {
+          const uint4 *src =
+              reinterpret_cast<const uint4 *>(smem + C::kOffSfa + slot * C::kSfa) + lane;
+          if (Kd::kKGroups == 2) {
+            const uint4 g0 = src[0], g1 = src[32];
+            const uint32_t r[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            tc_st_x8(dst, r);
+          } else {
+            const uint4 g0 = src[0];
+            const uint32_t r[4] = {g0.x, g0.y, g0.z, g0.w};
+            tc_st_x4(dst, r);
+          }
+          if (!Kd::kRowScaledB) {
+            // kind::mxf8f6f4's B block scales: the same layout, one 128-row
+            // chunk of B after another, behind the A scale columns
+            const uint4 *srb =
+                reinterpret_cast<const uint4 *>(smem + C::kOffSfb + slot * C::kSfb) + lane;
+#pragma unroll
+            for (int gc = 0; gc < Kd::kKGroups * C::kRowChunks; ++gc) {
+              const uint4 v = srb[32 * gc];
+              const uint32_t r[4] = {v.x, v.y, v.z, v.w};
+              tc_st_x4(dst + 4 * Kd::kKGroups + 4 * gc, r);
+            }
           }
         }
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (C::kSfRing) {
+        if (sft) {
+          if (++sub == C::kSfGroup) sub = 0;
+        } else if (C::kSfRing) {
           // the slot's bytes are in registers and stored: the loader may refill it
           if (lane == 0) mbar_arrive(&sfs_empty[slot]);
           if (++slot == C::kSfSlots) { slot = 0; sph ^= 1; }
@@ -1656,10 +1771,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     if (warp == 0 && lane == 0)
       for (int j = max(0, issued - C::kStages); j < issued; ++j)
         mbar_wait_drain(&full[j % C::kStages], (uint32_t)(j / C::kStages) & 1u);
-    // the scale loader's last signals: their cp.async arrivals have landed
+    // the scale loader's last signals: their cp.async arrivals or TMA bytes
+    // have landed
     if (warp == 1)
-      for (int j = max(0, l_signaled - C::kSfSlots); j < l_signaled; ++j)
-        mbar_wait_drain(&sfs_full[j % C::kSfSlots], (uint32_t)(j / C::kSfSlots) & 1u);
+      for (int j = max(0, l_signaled - n_sfslots); j < l_signaled; ++j)
+        mbar_wait_drain(&sfs_full[j % n_sfslots], (uint32_t)(j / n_sfslots) & 1u);
     __syncthreads();
   }
   if (PAIR) {
@@ -1739,9 +1855,11 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // 2-D K-major tensor map: inner dimension `inner` elements, `rows` rows,
-// row pitch `pitch` bytes, box `box_inner` x `box_rows`, 128-byte swizzle.
+// row pitch `pitch` bytes, box `box_inner` x `box_rows`, 128-byte swizzle
+// (or none: the 16-byte scale groups).
 inline bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
-                     uint64_t rows, uint64_t pitch, uint32_t box_inner, uint32_t box_rows) {
+                     uint64_t rows, uint64_t pitch, uint32_t box_inner, uint32_t box_rows,
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, rows};
@@ -1749,8 +1867,10 @@ inline bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, u
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            swz == CU_TENSOR_MAP_SWIZZLE_NONE ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                              : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Weight map of one matrix [E*rows, K]: padded E2M1 (box 128 elements) for
@@ -1821,12 +1941,13 @@ inline int tc_pair_grid(int sms) {
 // here instead of encoding twelve maps on the host per call.  A handful of
 // entries, replaced round-robin, under a mutex.
 struct TcMapKey {
-  int kind, bn, dev, H, I, E;
+  int kind, bn, pair, dev, H, I, E;
   size_t P;
-  const void *w13c, *w2c, *xq, *hq;
+  const void *w13c, *w2c, *w13s, *w2s, *xq, *hq;
   bool operator==(const TcMapKey &o) const {
-    return kind == o.kind && bn == o.bn && dev == o.dev && H == o.H && I == o.I && E == o.E &&
-           P == o.P && w13c == o.w13c && w2c == o.w2c && xq == o.xq && hq == o.hq;
+    return kind == o.kind && bn == o.bn && pair == o.pair && dev == o.dev && H == o.H &&
+           I == o.I && E == o.E && P == o.P && w13c == o.w13c && w2c == o.w2c &&
+           w13s == o.w13s && w2s == o.w2s && xq == o.xq && hq == o.hq;
   }
 };
 
@@ -1927,9 +2048,14 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   a2.K = I;
   a2.rows_per_expert = H;
   a2.tile_counter = counters + 1;
+  // scale bytes by TMA: 16-byte groups of whole rows (K % 512 == 0) from
+  // 16-byte aligned scale arrays
+  auto al16 = [](const void *q) { return ((uintptr_t)q & 15u) == 0; };
+  a1.sf_tma = KIND == KIND_F8 && H % 512 == 0 && al16(f.w13s) ? 1 : 0;
+  a2.sf_tma = KIND == KIND_F8 && I % 512 == 0 && al16(f.w2s) ? 1 : 0;
 
-  TcMaps maps1, maps2;
-  const TcMapKey key{KIND, BN, dev, H, I, E, P, f.w13c, f.w2c, xq, hq};
+  TcMaps maps1{}, maps2{};
+  const TcMapKey key{KIND, BN, PAIR, dev, H, I, E, P, f.w13c, f.w2c, f.w13s, f.w2s, xq, hq};
   if (!tc_map_cache().find(key, maps1, maps2)) {
     if (!make_weight_map<KIND>(&maps1.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
     for (int i = 0; i < 4; ++i)
@@ -1941,6 +2067,25 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
       if (!make_map(&maps2.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hq, hrow, T * P, hrow, 128,
                     a1.b_box[i]))
         return MOE_ERR_CUDA;
+    const auto nosw = CU_TENSOR_MAP_SWIZZLE_NONE;
+    if (a1.sf_tma) {
+      if (!make_map(&maps1.sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, f.w13s, H / 32, (uint64_t)E * 2 * I,
+                    H / 32, 16, 64, nosw))
+        return MOE_ERR_CUDA;
+      for (int i = 0; i < 4; ++i)
+        if (!make_map(&maps1.sb[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xs, H / 32, T * P, H / 32, 16,
+                      a1.b_box[i], nosw))
+          return MOE_ERR_CUDA;
+    }
+    if (a2.sf_tma) {
+      if (!make_map(&maps2.sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, f.w2s, I / 32, (uint64_t)E * H,
+                    I / 32, 16, 64, nosw))
+        return MOE_ERR_CUDA;
+      for (int i = 0; i < 4; ++i)
+        if (!make_map(&maps2.sb[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hs, I / 32, T * P, I / 32, 16,
+                      a1.b_box[i], nosw))
+          return MOE_ERR_CUDA;
+    }
     tc_map_cache().put(key, maps1, maps2);
   }
 

@@ -218,6 +218,11 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -815,9 +820,9 @@ struct TcCfg {
   // ahead; sized to leave the operand stages as many as before.  Else one
   // scale slot per operand stage.
   static constexpr int kSfRing = KIND == KIND_F8 ? (PAIR ? 8 : 4) : 0;
-  // With TcArgs::sf_tma the scale bytes come instead in groups of kSfGroup
-  // stages (16 bytes of each A and B row) by TMA, into one of kSftSlots
-  // slots of [128 A rows][16] then [BN B rows][16] bytes.
+  // With TcArgs::sf_tma (kind::mxf8f6f4) the scale bytes come instead in
+  // groups of kSfGroup stages (16 bytes of each A and B row) by TMA, into one
+  // of kSftSlots slots of [128 A rows][16] then [BN B rows][16] bytes.
   static constexpr int kSfGroup = 16 / (4 * Kd::kKGroups);
   static constexpr int kSftA = 128 * 16;               // A part of a slot; the B part follows
   static constexpr int kSft = KIND == KIND_F8 ? kSftA + 16 * BN : 0;   // all B rows (PAIR too)
@@ -1225,10 +1230,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     if (sft) {
       // 16 bytes of every A row and B row of the tile -- the scale bytes of
       // kSfGroup stages -- per TMA group: the two 64-row halves of the weight
-      // tile, then the B tile's boxes (evict-first and evict-last, as their
-      // operands), into a slot of [row][16] bytes.  The writer warps free a
-      // slot as soon as they have read it, at the group's first stage.
-      const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+      // tile, then the B tile's boxes, into a slot of [row][16] bytes.  A row's
+      // later groups read the rest of the line its first group brought into
+      // L2, so the weight scales are not marked evict-first as the weights
+      // are.  The writer warps free a slot as soon as they have read it, at
+      // the group's first stage.
+      const uint64_t pol_w = policy_evict_normal(), pol_x = policy_evict_last();
       int slot = 0;
       uint32_t sph = 0;
       bool ok = true;
@@ -1236,8 +1243,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         const int t = ring_read(ring_full, ring_empty, ring, ti, lane == 0, abort, n_tiles);
         if (!__all_sync(FULL, t < n_tiles && !*abort)) break;
         const Tile tl = decode(t);
-        const int arow = tl.e * a.rows_per_expert + (MODE == 1 ? tl.mt * 64 : tl.mt * 128);
-        const int arow2 = arow + (MODE == 1 ? a.I : 64);
+        const TcArgs &ap = tl.ph ? a2 : a;       // this phase's operands
+        const TcMaps &mp = tl.ph ? maps2 : maps;
+        const bool m1 = mode_of(tl.ph) == 1;
+        const int arow = tl.e * ap.rows_per_expert + (m1 ? tl.mt * 64 : tl.mt * 128);
+        const int arow2 = arow + (m1 ? a.I : 64);
         const int bsel = b_box_sel((tl.nB + 15) & ~15);
         const int tail = bsel >> 3;
         const uint32_t bytes =
@@ -1251,12 +1261,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           if (lane == 0) {
             uint8_t *dst = smem + C::kOffSfa + slot * C::kSft;
             mbar_expect_tx(&sfs_full[slot], bytes);
-            tma_load_2d(dst, &maps.sa, 16 * gi, arow, &sfs_full[slot], pol_w);
-            tma_load_2d(dst + 64 * 16, &maps.sa, 16 * gi, arow2, &sfs_full[slot], pol_w);
-            tma_load_2d(dst + C::kSftA, &maps.sb[bsel & 7], 16 * gi, tl.rowB, &sfs_full[slot],
+            tma_load_2d(dst, &mp.sa, 16 * gi, arow, &sfs_full[slot], pol_w);
+            tma_load_2d(dst + 64 * 16, &mp.sa, 16 * gi, arow2, &sfs_full[slot], pol_w);
+            tma_load_2d(dst + C::kSftA, &mp.sb[bsel & 7], 16 * gi, tl.rowB, &sfs_full[slot],
                         pol_x);
             if (tail)
-              tma_load_2d(dst + C::kSftA + 128 * 16, &maps.sb[tail - 1], 16 * gi, tl.rowB + 128,
+              tma_load_2d(dst + C::kSftA + 128 * 16, &mp.sb[tail - 1], 16 * gi, tl.rowB + 128,
                           &sfs_full[slot], pol_x);
           }
           ++l_signaled;
@@ -2051,6 +2061,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   // scale bytes by TMA: 16-byte groups of whole rows (K % 512 == 0) from
   // 16-byte aligned scale arrays
   auto al16 = [](const void *q) { return ((uintptr_t)q & 15u) == 0; };
+  // (kind::mxf4 keeps its cp.async scale loads: with TMA the HBM-bound
+  // kind::mxf4 GEMMs measured 1.3-2 % slower)
   a1.sf_tma = KIND == KIND_F8 && H % 512 == 0 && al16(f.w13s) ? 1 : 0;
   a2.sf_tma = KIND == KIND_F8 && I % 512 == 0 && al16(f.w2s) ? 1 : 0;
 

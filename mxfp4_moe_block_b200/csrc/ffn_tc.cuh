@@ -213,6 +213,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
+// 3-D box: c0 innermost
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1,
+                                            int c2, uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -766,10 +776,14 @@ inline cudaError_t launch_encode_f4(const uint16_t *src, const int32_t *sp, int 
 // ------------------------------------------------------------- the kernel --
 
 struct TcMaps {
-  CUtensorMap a;        // weights [E*rows, K]: box 128 (padded E2M1) or 128 B (packed) x 64 rows
+  // weights, box 128 (padded E2M1) or 128 B (packed) wide: GEMM-1's [E*2I, K]
+  // as [2E][I][K], a box of 64 rows of both halves (gate, then up); GEMM-2's
+  // [E*H, K], a box of 128 rows -- one TMA per stage either way
+  CUtensorMap a;
   CUtensorMap b[4];     // activation terms [T*P, row bytes]: box 128 B x {16, 32, 64, 128} rows
-  // scale bytes in 16-byte groups (TcArgs::sf_tma): weights [E*rows, K/32],
-  // box 16 B x 64 rows; activation terms [T*P, K/32], box 16 B x the B boxes' rows
+  // scale bytes in 16-byte groups (TcArgs::sf_tma): weights [E*rows, K/32]
+  // (16 B of the same rows as map a); activation terms [T*P, K/32], box 16 B
+  // x the B boxes' rows
   CUtensorMap sa;
   CUtensorMap sb[4];
 };
@@ -1112,7 +1126,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       // rows more than the tile's N.  PAIR: N rounded up to 32, this CTA's
       // half (a multiple of 16 rows) in one box of up to 64 rows or a 64-row
       // box and a second one.
-      auto tile_geom = [&](int t, int &arow, int &rowB, int &bsel, int &ph, int &g) {
+      auto tile_geom = [&](int t, int &ac1, int &ac2, int &rowB, int &bsel, int &ph, int &g) {
         const Tile tl = decode(t);
         if (PAIR) {
           const int half = ((tl.nB + 31) & ~31) / 2;
@@ -1125,21 +1139,25 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         ph = tl.ph;
         g = tl.g;
         const int rpe = ph ? a2.rows_per_expert : a.rows_per_expert;
-        arow = tl.e * rpe + (mode_of(ph) == 1 ? tl.mt * 64 : tl.mt * 128);
+        // the weight box: GEMM-1 rows m*64.. of halves 2e, 2e + 1; GEMM-2 rows
+        // e*H + m*128..
+        ac1 = mode_of(ph) == 1 ? tl.mt * 64 : tl.e * rpe + tl.mt * 128;
+        ac2 = 2 * tl.e;
       };
       auto b_bytes = [&](int bsel) {
         const int tail = bsel >> 3;
         return (uint32_t)(a.b_box[bsel & 7] + (tail ? a.b_box[tail - 1] : 0)) * 128u;
       };
       // the box's inner coordinate is in elements (padded E2M1) or bytes
-      // (packed E2M1); both are kt * 128.  Rows 0-63 of the tile, then rows
-      // 64-127 (GEMM-1: gate, then up).
-      auto load_a = [&](int st, int arow, int kt, int ph) {
+      // (packed E2M1); both are kt * 128.  One box of the tile's 128 rows
+      // (GEMM-1: 64 gate rows, then 64 up rows)
+      auto load_a = [&](int st, int ac1, int ac2, int kt, int ph) {
         uint8_t *sa = smem + st * C::kA;
         const CUtensorMap *m = ph ? &maps2.a : &maps.a;
-        tma_load_2d(sa, m, kt * 128, arow, &full[st], pol_w);
-        tma_load_2d(sa + 64 * 128, m, kt * 128, arow + (mode_of(ph) == 1 ? a.I : 64), &full[st],
-                    pol_w);
+        if (mode_of(ph) == 1)
+          tma_load_3d(sa, m, kt * 128, ac1, ac2, &full[st], pol_w);
+        else
+          tma_load_2d(sa, m, kt * 128, ac1, &full[st], pol_w);
       };
       auto load_b = [&](int st, int bsel, int rowB, int kt, int ph) {
         uint8_t *sb = smem + C::kOffB + st * C::kB;
@@ -1180,12 +1198,12 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
       // of A stream in before the wait for the activation operand.
       int npre = 0;
       if (pair_id < n_tiles) {
-        int arow, rowB, bsel, ph, g;
-        tile_geom(pair_id, arow, rowB, bsel, ph, g);
+        int ac1, ac2, rowB, bsel, ph, g;
+        tile_geom(pair_id, ac1, ac2, rowB, bsel, ph, g);
         npre = min(C::kStages, ksteps_of(ph));
         for (int kt = 0; kt < npre; ++kt) {
           mbar_expect_tx(&full[kt], Kd::kABytes + b_bytes(bsel));
-          load_a(kt, arow, kt, ph);
+          load_a(kt, ac1, ac2, kt, ph);
         }
         pdl_wait();
         pdl_trigger();
@@ -1202,15 +1220,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         // the next tile, published before this one's stages are issued
         const int t_next = PAIR ? t + n_units : n_units + atomicAdd(a.tile_counter, 1);
         if (!publish(t_next < n_tiles ? t_next : n_tiles)) break;
-        int arow, rowB, bsel, ph, g;
-        tile_geom(t, arow, rowB, bsel, ph, g);
+        int ac1, ac2, rowB, bsel, ph, g;
+        tile_geom(t, ac1, ac2, rowB, bsel, ph, g);
         const uint32_t bbytes = b_bytes(bsel);
         if (t != pair_id && !b_ready(ph, g)) break;
         const int ksteps = ksteps_of(ph);
         for (int kt = t == pair_id ? npre : 0; kt < ksteps; ++kt) {
           if (!mbar_wait_fast(&empty[stage], phase ^ 1, abort)) break;
           mbar_expect_tx(&full[stage], Kd::kABytes + bbytes);
-          load_a(stage, arow, kt, ph);
+          load_a(stage, ac1, ac2, kt, ph);
           load_b(stage, bsel, rowB, kt, ph);
           ++issued;
           if (++stage == C::kStages) { stage = 0; phase ^= 1; }
@@ -1229,8 +1247,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     if (!Kd::kRowScaledB) pdl_wait();        // B block scales come from the previous kernel
     if (sft) {
       // 16 bytes of every A row and B row of the tile -- the scale bytes of
-      // kSfGroup stages -- per TMA group: the two 64-row halves of the weight
-      // tile, then the B tile's boxes, into a slot of [row][16] bytes.  A row's
+      // kSfGroup stages -- per TMA group: the weight tile's 128 rows, then the
+      // B tile's boxes, into a slot of [row][16] bytes.  A row's
       // later groups read the rest of the line its first group brought into
       // L2, so the weight scales are not marked evict-first as the weights
       // are.  The writer warps free a slot as soon as they have read it, at
@@ -1246,8 +1264,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
         const TcArgs &ap = tl.ph ? a2 : a;       // this phase's operands
         const TcMaps &mp = tl.ph ? maps2 : maps;
         const bool m1 = mode_of(tl.ph) == 1;
-        const int arow = tl.e * ap.rows_per_expert + (m1 ? tl.mt * 64 : tl.mt * 128);
-        const int arow2 = arow + (m1 ? a.I : 64);
+        const int arow = m1 ? tl.mt * 64 : tl.e * ap.rows_per_expert + tl.mt * 128;
         const int bsel = b_box_sel((tl.nB + 15) & ~15);
         const int tail = bsel >> 3;
         const uint32_t bytes =
@@ -1261,8 +1278,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
           if (lane == 0) {
             uint8_t *dst = smem + C::kOffSfa + slot * C::kSft;
             mbar_expect_tx(&sfs_full[slot], bytes);
-            tma_load_2d(dst, &mp.sa, 16 * gi, arow, &sfs_full[slot], pol_w);
-            tma_load_2d(dst + 64 * 16, &mp.sa, 16 * gi, arow2, &sfs_full[slot], pol_w);
+            if (m1)   // the weight tile's rows, as map a: 64 gate, then 64 up
+              tma_load_3d(dst, &mp.sa, 16 * gi, arow, 2 * tl.e, &sfs_full[slot], pol_w);
+            else
+              tma_load_2d(dst, &mp.sa, 16 * gi, arow, &sfs_full[slot], pol_w);
             tma_load_2d(dst + C::kSftA, &mp.sb[bsel & 7], 16 * gi, tl.rowB, &sfs_full[slot],
                         pol_x);
             if (tail)
@@ -1883,13 +1902,44 @@ inline bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Weight map of one matrix [E*rows, K]: padded E2M1 (box 128 elements) for
-// kind::mxf8f6f4, packed bytes (box 128 bytes = 256 codes) for kind::mxf4.
+// 3-D map: [outer][mid][inner], pitches `pitch` (mid) and `pitch2` (outer)
+// bytes, box `box_inner` x `box_mid` x `box_outer`.
+inline bool make_map3(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                      uint64_t mid, uint64_t outer, uint64_t pitch, uint64_t pitch2,
+                      uint32_t box_inner, uint32_t box_mid, uint32_t box_outer,
+                      CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {pitch, pitch2};
+  const cuuint32_t box[3] = {box_inner, box_mid, box_outer};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            swz == CU_TENSOR_MAP_SWIZZLE_NONE ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                              : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Weight maps: padded E2M1 (box 128 elements) for kind::mxf8f6f4, packed
+// bytes (box 128 bytes = 256 codes) for kind::mxf4.  GEMM-1's [E*2I, K] as
+// [2E][I][K] with a box of 64 rows x both halves of one expert (its gate and
+// up rows of the tile); GEMM-2's [E*H, K] with a box of 128 rows.
+template <int KIND>
+inline bool make_weight_map_gate_up(CUtensorMap *m, const uint8_t *codes, uint64_t K, uint64_t I,
+                                    uint64_t E) {
+  const uint64_t pitch = K / 2;
+  if (KIND == KIND_F4)
+    return make_map3(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, I, 2 * E, pitch, I * pitch,
+                     128, 64, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map3(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, codes, K, I, 2 * E, pitch,
+                   I * pitch, 128, 64, 2, CU_TENSOR_MAP_SWIZZLE_128B);
+}
 template <int KIND>
 inline bool make_weight_map(CUtensorMap *m, const uint8_t *codes, uint64_t K, uint64_t rows) {
   if (KIND == KIND_F4)
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, rows, K / 2, 128, 64);
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, codes, K, rows, K / 2, 128, 64);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, rows, K / 2, 128, 128);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, codes, K, rows, K / 2, 128, 128);
 }
 
 // Maximum dynamic shared memory of the two GEMM kernels of one
@@ -2069,7 +2119,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
   TcMaps maps1{}, maps2{};
   const TcMapKey key{KIND, BN, PAIR, dev, H, I, E, P, f.w13c, f.w2c, f.w13s, f.w2s, xq, hq};
   if (!tc_map_cache().find(key, maps1, maps2)) {
-    if (!make_weight_map<KIND>(&maps1.a, f.w13c, H, (uint64_t)E * 2 * I)) return MOE_ERR_CUDA;
+    if (!make_weight_map_gate_up<KIND>(&maps1.a, f.w13c, H, I, E)) return MOE_ERR_CUDA;
     for (int i = 0; i < 4; ++i)
       if (!make_map(&maps1.b[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, xrow, T * P, xrow, 128,
                     a1.b_box[i]))
@@ -2081,8 +2131,8 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
         return MOE_ERR_CUDA;
     const auto nosw = CU_TENSOR_MAP_SWIZZLE_NONE;
     if (a1.sf_tma) {
-      if (!make_map(&maps1.sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, f.w13s, H / 32, (uint64_t)E * 2 * I,
-                    H / 32, 16, 64, nosw))
+      if (!make_map3(&maps1.sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, f.w13s, H / 32, I, 2 * (uint64_t)E,
+                     H / 32, (uint64_t)I * (H / 32), 16, 64, 2, nosw))
         return MOE_ERR_CUDA;
       for (int i = 0; i < 4; ++i)
         if (!make_map(&maps1.sb[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, xs, H / 32, T * P, H / 32, 16,
@@ -2091,7 +2141,7 @@ int tc_run(const FfnArgs &f, uint8_t *ws, int sms, cudaStream_t s) {
     }
     if (a2.sf_tma) {
       if (!make_map(&maps2.sa, CU_TENSOR_MAP_DATA_TYPE_UINT8, f.w2s, I / 32, (uint64_t)E * H,
-                    I / 32, 16, 64, nosw))
+                    I / 32, 16, 128, nosw))
         return MOE_ERR_CUDA;
       for (int i = 0; i < 4; ++i)
         if (!make_map(&maps2.sb[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, hs, I / 32, T * P, I / 32, 16,

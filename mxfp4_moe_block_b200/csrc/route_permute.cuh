@@ -92,6 +92,8 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
 
   for (int e = lane; e < E; e += 32) cnt[w * E + e] = 0;
   __syncwarp();
+  // bits of an expert id or of the no-expert key E
+  const int kbits = 32 - __clz(E);
   // pass A.  The lane's expert ids for PERM_BATCH steps of 32 pairs are
   // loaded first (independent loads in flight), then ranked step by step.
   for (int b0 = p0; b0 < p1; b0 += 32 * PERM_BATCH) {
@@ -103,16 +105,16 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
     }
 #pragma unroll
     for (int j = 0; j < PERM_BATCH; ++j) {
+      if (b0 + 32 * j >= p1) break;          // warp-uniform: the range has ended
       const int p = b0 + 32 * j + lane;
       int e = ev[j];
       if (p < p1 && (e < 0 || e >= E)) { raise_status(MOE_DEV_BAD_EXPERT); e = -1; }
       if (p >= p1) e = -1;
-      // lanes holding the same expert: the bits of e (-1 taken as 1024, E <=
-      // 1024) by ballots -- 11 ballots cost less than __match_any_sync here
-      const unsigned key = e < 0 ? 1024u : (unsigned)e;
+      // lanes holding the same expert: the bits of e (-1 taken as E) by
+      // ballots -- cheaper than __match_any_sync here
+      const unsigned key = e < 0 ? (unsigned)E : (unsigned)e;
       unsigned same = FULL;
-#pragma unroll
-      for (int bit = 0; bit < 11; ++bit) {
+      for (int bit = 0; bit < kbits; ++bit) {
         const unsigned bb = __ballot_sync(FULL, (key >> bit) & 1u);
         same &= ((key >> bit) & 1u) ? bb : ~bb;
       }
@@ -174,6 +176,7 @@ __device__ __forceinline__ void permute_block(const int32_t *topk_idx, int P, in
     }
 #pragma unroll
     for (int j = 0; j < PERM_BATCH; ++j) {
+      if (b0 + 32 * j >= p1) break;
       const int p = b0 + 32 * j + lane;
       const int e = ev[j];
       if (p < p1 && e >= 0 && e < E) {

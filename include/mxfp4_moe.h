@@ -146,6 +146,10 @@ int moe_route_permute(const float *logits, int T, int E, int k, int32_t *topk_id
  *                  mxfp4_moe_ffn_workspace_bytes(T, k, H, I) bytes, 256-byte
  *                  aligned; its contents on entry do not matter.
  *   Limits: H % 128 == 0, I % 128 == 0, 1 <= E <= 1024, 1 <= k <= 32.
+ *   The tensor-core variants load the code arrays by TMA: 16-byte aligned
+ *   (else MOE_ERR_CUDA).  Scale arrays of any alignment; where one is
+ *   16-byte aligned and its rows hold a multiple of 16 bytes (K % 512 == 0),
+ *   kind::mxf8f6f4 loads it by TMA as well (same results).
  *   The kernel variant: the tensor-core one wherever its limits allow
  *   (H >= 512), else the FMA one (see mxfp4_moe_ffn_variant).
  */

@@ -63,14 +63,25 @@ class EdgeLayer:
     def oracle_weights(self, e):
         return self.w13c[e], self.w13s[e], self.w2c[e], self.w2s[e]
 
-    def run(self, variant):
+    def run(self, variant, scale_offset=0):
+        """scale_offset: place both scale arrays that many bytes past a
+        16-byte boundary of device memory (the same bytes)."""
         sh = self.sh
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+        def t_at(a):
+            if not scale_offset:
+                return t(a)
+            buf = torch.zeros(a.size + 32, dtype=torch.uint8, device=DEV)
+            v = buf[scale_offset:scale_offset + a.size].view(a.shape)
+            v.copy_(t(a))
+            assert v.data_ptr() % 16 == scale_offset % 16
+            return v
         xb = synth.f32_to_bf16_bits(self.x.astype(np.float32))
         assert np.array_equal(synth.bf16_bits_to_f32(xb), self.x.astype(np.float32)), \
             "activations must be bf16 values"
         x = t(xb.view(np.int16)).view(torch.bfloat16)
-        w = [t(a) for a in (self.w13c, self.w13s, self.w2c, self.w2s)]
+        w = [t(self.w13c), t_at(self.w13s), t(self.w2c), t_at(self.w2s)]
         idx, tw = mm.moe_route_topk(t(self.logits), sh.k)
         off, sp, pr = mm.moe_permute(idx, sh.E)
         y, ws = mm.mxfp4_moe_ffn(x, sh.k, *w, off, sp, variant=variant)
@@ -186,3 +197,22 @@ def test_scale_matched_blocks_over_the_whole_e8m0_range():
     lo, hi = c & 0x0F, c >> 4
     L.w13c[:, :, big] = ((lo & 0x0B) | ((hi & 0x0B) << 4)).astype(np.uint8)   # |value| <= 1.5
     L.check([mm.FFN_FMA, mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F8_PAIR], "matched full E8M0")
+
+
+def test_mxf8f6f4_scale_bytes_by_tma_and_by_cp_async_agree():
+    """kind::mxf8f6f4 loads the scale bytes by TMA, 16 bytes of each row per
+    four stages, when K is a multiple of 512 and the scale arrays are 16-byte
+    aligned; else by 4-byte cp.async.  H = 1024 and I = 512 take the TMA path
+    for both GEMMs; the same scales 4 bytes off a 16-byte boundary take the
+    cp.async path.  Both give the same bits (the MMAs see the same operands)
+    and match the oracle; one-CTA and CTA-pair launches alike."""
+    sh = synth.Shape("sfpath", H=1024, I=512, E=16, k=4, S=2, K=8, V=64, seed=2106)
+    L = EdgeLayer(sh, empty=(2, 11))
+    _edge_values(L)
+    L.check([mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F8_PAIR], "scale path")
+    for v in (mm.FFN_TENSOR_F8, mm.FFN_TENSOR_F8_PAIR):
+        _, _, h_tma, y_tma = L.run(v)
+        _, _, h_cpa, y_cpa = L.run(v, scale_offset=4)
+        assert np.array_equal(h_tma, h_cpa), NAMES[v]
+        assert np.array_equal(y_tma, y_cpa), NAMES[v]
+        assert mm.moe_get_device_status() == (0, 0)

@@ -65,7 +65,10 @@ enum {
   MOE_DEV_BAD_EXPERT = 1,  /* moe_permute saw an expert id outside [0,E)   */
   MOE_DEV_NO_MASS = 2,     /* block_accept_rejection: target row all zero  */
   MOE_DEV_BAD_TOKEN = 3,   /* a draft token outside [0,V)                   */
-  MOE_DEV_TIMEOUT = 4      /* a bounded device wait ran out                */
+  MOE_DEV_TIMEOUT = 4,     /* a bounded device wait ran out                */
+  MOE_DEV_BAD_INDEX = 5    /* checked build (MOE_CHECKS): a pair, row or
+                              offset index outside its array, replaced by 0
+                              or (offsets) the call's experts left empty   */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */

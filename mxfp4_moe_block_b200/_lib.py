@@ -13,11 +13,16 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmxfp4_moe.so")
+# MXFP4_MOE_CHECKS=1: the checked build (every caller-supplied index tested
+# on the device before use; see build.py)
+LIB_PATH = os.path.join(HERE, "libmxfp4_moe_checks.so" if os.environ.get("MXFP4_MOE_CHECKS") == "1"
+                        else "libmxfp4_moe.so")
 
 MOE_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "CUDA error",
                 4: "workspace", 5: "device status"}
+# device status details (second value of moe_get_device_status)
+DEV_OK, DEV_BAD_EXPERT, DEV_NO_MASS, DEV_BAD_TOKEN, DEV_TIMEOUT, DEV_BAD_INDEX = 0, 1, 2, 3, 4, 5
 (FFN_AUTO, FFN_FMA, FFN_TENSOR, FFN_TENSOR_F8, FFN_TENSOR_F4, FFN_TENSOR_FUSED,
  FFN_TENSOR_F8_PAIR) = 0, 1, 2, 3, 4, 5, 6
 
@@ -68,7 +73,8 @@ def lib() -> ctypes.CDLL:
     if _LIB is None:
         if not os.path.exists(LIB_PATH):
             raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m mxfp4_moe_block_b200.build`")
+                f"{LIB_PATH} is missing: build it with `python -m mxfp4_moe_block_b200.build`"
+                + (" --checks" if LIB_PATH.endswith("_checks.so") else ""))
         L = ctypes.CDLL(LIB_PATH)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(L, name)

@@ -1,8 +1,12 @@
 """Build the CUDA library in-tree: libmxfp4_moe.so next to this file.
 
-    python -m mxfp4_moe_block_b200.build
+    python -m mxfp4_moe_block_b200.build            # libmxfp4_moe.so
+    python -m mxfp4_moe_block_b200.build --checks   # libmxfp4_moe_checks.so
 
 Compiles csrc/mxfp4_moe.cu (which includes every kernel) for sm_100a only.
+The checked build (-DMOE_CHECKS) tests every index read from a caller's
+array before it addresses memory and reports a bad one in the device status
+word (MOE_DEV_BAD_INDEX); the package loads it when MXFP4_MOE_CHECKS=1.
 """
 import os
 import subprocess
@@ -11,6 +15,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "csrc", "mxfp4_moe.cu")
 OUT = os.path.join(HERE, "libmxfp4_moe.so")
+OUT_CHECKS = os.path.join(HERE, "libmxfp4_moe_checks.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -28,25 +33,25 @@ def sources():
         os.path.join(os.path.dirname(HERE), "include", "mxfp4_moe.h")]
 
 
-def up_to_date():
-    if not os.path.exists(OUT):
+def up_to_date(out=OUT):
+    if not os.path.exists(out):
         return False
-    t = os.path.getmtime(OUT)
+    t = os.path.getmtime(out)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force=False, verbose=False):
-    if not force and up_to_date():
-        return OUT
-    cmd = [NVCC, *FLAGS, "-o", OUT + ".tmp", SRC]
+def build(force=False, verbose=False, checks=False):
+    out = OUT_CHECKS if checks else OUT
+    if not force and up_to_date(out):
+        return out
+    cmd = [NVCC, *FLAGS, *(["-DMOE_CHECKS"] if checks else []), "-o", out + ".tmp", SRC]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(OUT + ".tmp", OUT)
-    return OUT
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="-v" in sys.argv)
-    print(OUT)
+    print(build(force=True, verbose="-v" in sys.argv, checks="--checks" in sys.argv))

@@ -22,7 +22,8 @@ combine_kernel(const float *__restrict__ y, const int32_t *__restrict__ pair_row
   __shared__ const float *rows[32];
   __shared__ float wts[32];
   if (threadIdx.x < k) {
-    rows[threadIdx.x] = y + (size_t)__ldg(pair_row + (size_t)t * k + threadIdx.x) * H;
+    rows[threadIdx.x] =
+        y + (size_t)checked_index(__ldg(pair_row + (size_t)t * k + threadIdx.x), (long)T * k) * H;
     wts[threadIdx.x] = __ldg(topk_w + (size_t)t * k + threadIdx.x);
   }
   __syncthreads();

@@ -22,6 +22,40 @@ __device__ __forceinline__ void raise_status(int detail) {
   atomicCAS(&g_status, 0, detail);
 }
 
+// Checked build (-DMOE_CHECKS, libmxfp4_moe_checks.so): every index read
+// from a caller's array -- the pair ids of sorted_pair and pair_row, the
+// expert offsets -- is checked before it addresses memory; a bad one sets
+// MOE_DEV_BAD_INDEX and is replaced by 0 (offsets: the call's experts are
+// left empty).  No trap, no access outside the arrays.  Off in the normal
+// build, where those arrays are trusted to come from moe_permute.
+#ifdef MOE_CHECKS
+constexpr bool kChecks = true;
+__device__ __forceinline__ int checked_index(int i, long n) {
+  if (i < 0 || i >= n) {
+    raise_status(MOE_DEV_BAD_INDEX);
+    return 0;
+  }
+  return i;
+}
+#else
+constexpr bool kChecks = false;
+__device__ __forceinline__ int checked_index(int i, long) { return i; }
+#endif
+
+// Checked build: expert offsets off[0..E] non-decreasing from >= 0 to <= P,
+// tested by one warp (all lanes get the verdict); false sets MOE_DEV_BAD_INDEX.
+__device__ __forceinline__ bool offsets_ok(const int32_t *off, int E, long P) {
+  if (!kChecks) return true;
+  bool bad = false;
+  for (int e = (int)(threadIdx.x & 31); e < E; e += 32) {
+    const int a = __ldg(off + e), b = __ldg(off + e + 1);
+    bad |= a < 0 || b < a || b > P;
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad && (threadIdx.x & 31) == 0) raise_status(MOE_DEV_BAD_INDEX);
+  return !bad;
+}
+
 constexpr unsigned FULL = 0xffffffffu;
 
 // Programmatic dependent launch.  Every kernel of the library is launched

@@ -62,11 +62,12 @@ x_to_f32_kernel(const uint16_t *__restrict__ x, size_t n8, float *__restrict__ x
 
 // Active-expert list of one CTA: experts with at least one row, ascending.
 // Built by warp 0; returns the count after a __syncthreads.
-__device__ __forceinline__ int build_active(const int32_t *__restrict__ off, int E,
+__device__ __forceinline__ int build_active(const int32_t *__restrict__ off, int E, long P,
                                             int *s_act, int *s_n) {
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     int n = 0;
+    if (!offsets_ok(off, E, P)) E = 0;           // checked build: bad offsets, no work
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       const bool on = e < E && __ldg(off + e + 1) > __ldg(off + e);
@@ -155,7 +156,7 @@ __device__ __forceinline__ void ffn1_group(const FfnArgs &a, int e, int n0, int 
   const float *xr[NT];
 #pragma unroll
   for (int j = 0; j < NT; ++j)
-    xr[j] = a.x32 + (size_t)(__ldg(a.sp + r0 + t0 + j) / a.k) * a.H;
+    xr[j] = a.x32 + (size_t)(checked_index(__ldg(a.sp + r0 + t0 + j), (long)a.T * a.k) / a.k) * a.H;
   float acc[2 * RG][NT];
   fma_rows<2 * RG, NT>(a.w13c + erows * (a.H / 2), a.w13s + erows * (a.H / 32), rowoff, a.H,
                        xr, lane, acc);
@@ -180,7 +181,7 @@ ffn1_fma_kernel(FfnArgs a) {
   pdl_trigger();
   __shared__ int s_act[1024];
   __shared__ int s_n;
-  const int n_act = build_active(a.off, a.E, s_act, &s_n);
+  const int n_act = build_active(a.off, a.E, (long)a.T * a.k, s_act, &s_n);
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -226,7 +227,7 @@ ffn2_fma_kernel(FfnArgs a) {
   pdl_trigger();
   __shared__ int s_act[1024];
   __shared__ int s_n;
-  const int n_act = build_active(a.off, a.E, s_act, &s_n);
+  const int n_act = build_active(a.off, a.E, (long)a.T * a.k, s_act, &s_n);
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;

@@ -562,7 +562,7 @@ split_x_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ sp, i
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
        i += (long)gridDim.x * blockDim.x) {
     const int r = (int)(i / nb), b = (int)(i % nb);
-    const int t = __ldg(sp + r) / k;
+    const int t = checked_index(__ldg(sp + r), P) / k;
     const uint16_t *src = x + (size_t)t * H + b * 32;
     float v[32];
     if (vec) {
@@ -612,7 +612,8 @@ encode_rows_f4_kernel(const uint16_t *__restrict__ src, const int32_t *__restric
     for (int i = threadIdx.x; i < ncounters; i += blockDim.x) counters[i] = 0;
   const int r = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const uint16_t *row = src + (size_t)(sp ? __ldg(sp + r) / k : r) * K;
+  const uint16_t *row =
+      src + (size_t)(sp ? checked_index(__ldg(sp + r), gridDim.x) / k : r) * K;
   __shared__ float red[ENC_THREADS / 32];
   const int npairs = K / 2;
   float v[2 * ENC_MAX_PAIRS];
@@ -671,7 +672,7 @@ encode_rows_f4_warp_kernel(const uint16_t *__restrict__ src, const int32_t *__re
   const int r = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (r >= P) return;
   const uint32_t *row =
-      reinterpret_cast<const uint32_t *>(src + (size_t)(sp ? __ldg(sp + r) / k : r) * K);
+      reinterpret_cast<const uint32_t *>(src + (size_t)(sp ? checked_index(__ldg(sp + r), P) / k : r) * K);
   float v[2 * PPL];
 #pragma unroll
   for (int j = 0; j < PPL; ++j) {
@@ -991,13 +992,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
   const bool sft = KIND == KIND_F8 && MODE != 3 && a.sf_tma != 0;
   const int n_sfslots = sft ? C::kSftSlots : C::kSfSlots;
 
-  // tile table: active experts and the prefix of their tile counts
+  // tile table: active experts and the prefix of their tile counts (none
+  // where the checked build finds the offsets bad)
   if (warp == 0) {
     int n = 0, acc = 0;
-    for (int e0 = 0; e0 < a.E; e0 += 32) {
+    const int n_e = offsets_ok(a.off, a.E, a.P) ? a.E : 0;
+    for (int e0 = 0; e0 < n_e; e0 += 32) {
       const int e = e0 + lane;
-      const int r0 = e < a.E ? __ldg(a.off + e) : 0;
-      const int cnt = e < a.E ? __ldg(a.off + e + 1) - r0 : 0;
+      const int r0 = e < n_e ? __ldg(a.off + e) : 0;
+      const int cnt = e < n_e ? __ldg(a.off + e + 1) - r0 : 0;
       const int nt = cnt > 0 ? (T * cnt + BN - 1) / BN : 0;
       const unsigned b = __ballot_sync(FULL, nt > 0);
       int sc = nt * mtiles;
@@ -1018,7 +1021,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcAr
     if (lane == 0) {
       s_act[1024] = (uint16_t)n;
       s_pre[n] = acc;
-      s_r0[n] = __ldg(a.off + a.E);   // rows of inactive experts are empty: the next
+      s_r0[n] = n_e ? __ldg(a.off + a.E) : 0;   // rows of inactive experts are empty: the next
                                        // active expert's first row ends the previous one
     }
   } else if (warp == 1 && lane == 0) {

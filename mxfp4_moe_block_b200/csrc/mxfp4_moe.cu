@@ -6,6 +6,8 @@
 #include <algorithm>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "route_permute.cuh"
 #include "ffn_fma.cuh"
@@ -19,6 +21,15 @@ using namespace moe;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// One NVTX range per C-ABI call, named after the call, for timeline tools
+// (a function-pointer check and nothing more when none is attached).
+struct CallRange {
+  explicit CallRange(const char *name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange &) = delete;
+  CallRange &operator=(const CallRange &) = delete;
+};
 
 struct DeviceInfo {
   bool ready = false;
@@ -119,6 +130,7 @@ static int permute_attributes() {
 // ------------------------------------------------------------------ route --
 int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
                    float *topk_w, moe_stream_t stream) {
+  const CallRange range("moe_route_topk");
   if (T < 0 || E < 1 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
@@ -137,6 +149,7 @@ int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_idx,
 // ---------------------------------------------------------------- permute --
 int moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *expert_offsets,
                 int32_t *sorted_pair, int32_t *pair_row, moe_stream_t stream) {
+  const CallRange range("moe_permute");
   if (T < 0 || k < 1 || k > 32 || E < 1) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
   const long long P = (long long)T * k;
@@ -154,6 +167,7 @@ int moe_permute(const int32_t *topk_idx, int T, int k, int E, int32_t *expert_of
 int moe_route_permute(const float *logits, int T, int E, int k, int32_t *topk_idx, float *topk_w,
                       int32_t *expert_offsets, int32_t *sorted_pair, int32_t *pair_row,
                       moe_stream_t stream) {
+  const CallRange range("moe_route_permute");
   if (T < 0 || E < 1 || k < 1 || k > E || k > 32) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
   if ((long long)T * k > (1ll << 24)) return MOE_ERR_UNSUPPORTED;
@@ -213,6 +227,7 @@ int mxfp4_moe_ffn_variant(const uint16_t *x, int T, int H, int I, int E, int k,
                           const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
                           void *workspace, size_t workspace_bytes, int variant,
                           moe_stream_t stream) {
+  const CallRange range("mxfp4_moe_ffn_variant");
   if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128) return MOE_ERR_INVALID_ARG;
   if (E > 1024) return MOE_ERR_UNSUPPORTED;
@@ -257,6 +272,7 @@ int mxfp4_moe_ffn(const uint16_t *x, int T, int H, int I, int E, int k,
                   const uint8_t *w2_codes, const uint8_t *w2_scales,
                   const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
                   void *workspace, size_t workspace_bytes, moe_stream_t stream) {
+  const CallRange range("mxfp4_moe_ffn");
   return mxfp4_moe_ffn_variant(x, T, H, I, E, k, w13_codes, w13_scales, w2_codes, w2_scales,
                                expert_offsets, sorted_pair, y, workspace, workspace_bytes,
                                MOE_FFN_AUTO, stream);
@@ -279,6 +295,7 @@ int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
                           const uint8_t *w2_codes, const uint8_t *w2_scales,
                           const int32_t *expert_offsets, const int32_t *sorted_pair, float *y,
                           moe_stream_t stream) {
+  const CallRange range("mxfp4_moe_ffn_noalloc");
   // the argument checks of mxfp4_moe_ffn_variant first, so that a bad
   // argument is reported as such whatever the problem's scratch need
   if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1 || k > 32 || k > E) return MOE_ERR_INVALID_ARG;
@@ -316,6 +333,7 @@ int mxfp4_moe_ffn_noalloc(const uint16_t *x, int T, int H, int I, int E, int k,
 // ---------------------------------------------------------------- combine --
 int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w, int T, int k,
                 int H, const uint16_t *residual, uint16_t *out, moe_stream_t stream) {
+  const CallRange range("moe_combine");
   if (T < 0 || k < 1 || k > 32 || H <= 0 || H % 8) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!y || !pair_row || !topk_w || !out) return MOE_ERR_INVALID_ARG;
@@ -326,6 +344,7 @@ int moe_combine(const float *y, const int32_t *pair_row, const float *topk_w, in
 
 int moe_rms_norm(const uint16_t *x, int T, int H, float eps, uint16_t *out,
                  moe_stream_t stream) {
+  const CallRange range("moe_rms_norm");
   if (T < 0 || H <= 0 || H % 8 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !out) return MOE_ERR_INVALID_ARG;
@@ -384,11 +403,13 @@ static int greedy_launch(const float *logits, const int32_t *draft, int S, int K
 
 int block_accept_greedy(const float *logits, const int32_t *draft, int S, int K, int V,
                         int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  const CallRange range("block_accept_greedy");
   return greedy_launch(logits, draft, S, K, V, K, accept_len, next_token, stream);
 }
 
 int block_accept_greedy_bonus(const float *logits, const int32_t *draft, int S, int K, int V,
                               int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  const CallRange range("block_accept_greedy_bonus");
   return greedy_launch(logits, draft, S, K, V, K + 1, accept_len, next_token, stream);
 }
 
@@ -409,6 +430,7 @@ static int rejection_launch(const float *p, const float *q, const int32_t *draft
 int block_accept_rejection(const float *p, const float *q, const int32_t *draft,
                            const float *u_accept, const float *u_resample, int S, int K, int V,
                            int32_t *accept_len, int32_t *next_token, moe_stream_t stream) {
+  const CallRange range("block_accept_rejection");
   return rejection_launch(p, q, draft, u_accept, u_resample, S, K, V, K, accept_len, next_token,
                           stream);
 }
@@ -417,6 +439,7 @@ int block_accept_rejection_bonus(const float *p, const float *q, const int32_t *
                                  const float *u_accept, const float *u_resample, int S, int K,
                                  int V, int32_t *accept_len, int32_t *next_token,
                                  moe_stream_t stream) {
+  const CallRange range("block_accept_rejection_bonus");
   return rejection_launch(p, q, draft, u_accept, u_resample, S, K, V, K + 1, accept_len,
                           next_token, stream);
 }
@@ -424,6 +447,7 @@ int block_accept_rejection_bonus(const float *p, const float *q, const int32_t *
 // --------------------------------------------------------------- quantise --
 int mxfp4_quantize(const uint16_t *w, int64_t R, int K, uint8_t *codes, uint8_t *scales,
                    moe_stream_t stream) {
+  const CallRange range("mxfp4_quantize");
   if (R < 0 || K < 32 || K % 32) return MOE_ERR_INVALID_ARG;
   if (R == 0) return MOE_OK;
   if (!w || !codes || !scales) return MOE_ERR_INVALID_ARG;

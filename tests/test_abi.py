@@ -79,3 +79,22 @@ def test_variant_range_is_checked(library):
     last = max(header_enum_values("MOE_FFN_").values())
     assert library.mxfp4_moe_ffn_variant(None, 1, 512, 256, 8, 2, None, None, None, None,
                                          None, None, None, None, 0, last + 1, None) == 1
+
+
+def test_device_detail_constants_match_the_header():
+    v = header_enum_values("MOE_DEV_")
+    assert v == {"MOE_DEV_OK": 0, "MOE_DEV_BAD_EXPERT": 1, "MOE_DEV_NO_MASS": 2,
+                 "MOE_DEV_BAD_TOKEN": 3, "MOE_DEV_TIMEOUT": 4, "MOE_DEV_BAD_INDEX": 5}
+    for name, val in v.items():
+        assert getattr(_lib, name[len("MOE_"):]) == val, name
+
+
+def test_checked_build_exports_every_declared_symbol():
+    """The MOE_CHECKS build (libmxfp4_moe_checks.so) is the same ABI."""
+    import ctypes
+    path = build.build(checks=True)
+    assert path.endswith("libmxfp4_moe_checks.so")
+    L = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    assert L.moe_version() == 10000

@@ -555,6 +555,40 @@ def cpu_baseline(sh):
 
 # ---------------------------------------------------------------------- e2e --
 
+def gpu_local_cpus(dev):
+    """The CPUs of the GPU's own NUMA node (its PCI device's local_cpulist in
+    sysfs) that this process may run on, or None where that is unknown."""
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        with open(f"/sys/bus/pci/devices/{bdf}/local_cpulist") as f:
+            text = f.read().strip()
+        cpus = set()
+        for part in text.split(","):
+            a, _, b = part.partition("-")
+            cpus.update(range(int(a), int(b or a) + 1))
+    except (AttributeError, OSError, ValueError):
+        return None
+    return (cpus & os.sched_getaffinity(0)) or None
+
+
+def pinned_near_gpu(n, dev):
+    """A pinned host buffer whose pages are placed on the GPU's NUMA node: the
+    allocating thread runs on that node's CPUs while the pages are allocated
+    and first written, then gets its former CPUs back (pages on a far node
+    would make every copy cross the socket link)."""
+    local, old = gpu_local_cpus(dev), os.sched_getaffinity(0)
+    if local:
+        os.sched_setaffinity(0, local)
+    try:
+        buf = torch.empty(n, dtype=torch.uint8).pin_memory()
+        buf.zero_()
+    finally:
+        if local:
+            os.sched_setaffinity(0, old)
+    return buf, (len(local) if local else None)
+
+
 def e2e_time(wl, variant, steps, warmup):
     """The same step through the public API with host buffers, as a serving
     loop runs it: every step's inputs (x, router logits, block logits, drafts;
@@ -570,11 +604,11 @@ def e2e_time(wl, variant, steps, warmup):
     for a in arrays:
         offs.append(o)
         o += (a.nbytes + 255) // 256 * 256
-    host_in = torch.empty(o, dtype=torch.uint8).pin_memory()
+    host_in, node_cpus = pinned_near_gpu(o, wl.dev)
     for a, off in zip(arrays, offs):
         host_in[off:off + a.nbytes] = torch.from_numpy(np.ascontiguousarray(a).reshape(-1))
     h2d = sum(a.nbytes for a in arrays)
-    host_out = torch.empty(wl.result.numel(), dtype=torch.uint8).pin_memory()
+    host_out, _ = pinned_near_gpu(wl.result.numel(), wl.dev)
     d2h = wl.result.numel()
     s = wl.sh_r
 
@@ -643,9 +677,9 @@ def e2e_time(wl, variant, steps, warmup):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
     # the host link alone: the step's input copy, and a large pinned copy
-    link = {}
+    link = {"host_buffers_on_gpu_node_cpus": node_cpus}
     for name, n in (("step_input", o), ("256MiB", 256 << 20)):
-        hsrc = host_in if n == o else torch.empty(n, dtype=torch.uint8).pin_memory()
+        hsrc = host_in if n == o else pinned_near_gpu(n, wl.dev)[0]
         dst = torch.empty(n, dtype=torch.uint8, device=wl.dev)
         with torch.cuda.stream(copy):
             for _ in range(3):

@@ -17,10 +17,13 @@
 // matrix, block of B rows): its first from blockIdx.x, the rest from an
 // atomic counter.  Warp roles, after the tile-pipelining and
 // warp-specialisation ideas the pages describe for TileRT (prior art):
-//   warp 0     TMA producer: weight tile + activation tile per 16 KB stage,
+//   warp 0     TMA producer: the weight tile (one box) and the activation tile
+//              of each stage,
 //              and the tile index ring every other role reads;
-//   warp 1     scale loader: cp.async of the scale bytes into shared memory
-//              in the 32-row x 16-byte layout of the scale-factor columns;
+//   warp 1     scale loader: the scale bytes into shared memory -- by TMA,
+//              16 bytes of each row per four stages (kind::mxf8f6f4, K a
+//              multiple of 512), else by cp.async in the 32-row x 16-byte
+//              layout of the scale-factor columns;
 //   warp 2     TMEM allocation and the single MMA-issuing thread;
 //   warp 3     constant B block scales (kind::mxf4);
 //   warps 4-7  epilogue: TMEM -> registers -> SwiGLU (GEMM-1) or y (GEMM-2);

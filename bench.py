@@ -555,6 +555,16 @@ def cpu_baseline(sh):
 
 # ---------------------------------------------------------------------- e2e --
 
+def parse_cpulist(text):
+    """CPU numbers of a Linux cpulist string ("0-3,8,10-11")."""
+    cpus = set()
+    for part in text.strip().split(","):
+        if part:
+            a, _, b = part.partition("-")
+            cpus.update(range(int(a), int(b or a) + 1))
+    return cpus
+
+
 def gpu_local_cpus(dev):
     """The CPUs of the GPU's own NUMA node (its PCI device's local_cpulist in
     sysfs) that this process may run on, or None where that is unknown."""
@@ -562,11 +572,7 @@ def gpu_local_cpus(dev):
         p = torch.cuda.get_device_properties(dev)
         bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
         with open(f"/sys/bus/pci/devices/{bdf}/local_cpulist") as f:
-            text = f.read().strip()
-        cpus = set()
-        for part in text.split(","):
-            a, _, b = part.partition("-")
-            cpus.update(range(int(a), int(b or a) + 1))
+            cpus = parse_cpulist(f.read())
     except (AttributeError, OSError, ValueError):
         return None
     return (cpus & os.sched_getaffinity(0)) or None

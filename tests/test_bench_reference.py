@@ -52,3 +52,13 @@ def test_l2_statement_follows_the_weight_bytes():
     from mxfp4_moe_block_b200 import synth
     assert bench.l2_statement(synth.SHAPES["batch1"]).startswith("inputs larger than L2")
     assert bench.l2_statement(synth.SHAPES["tiny"]).startswith("inputs smaller than L2")
+
+
+def test_cpulist_parser():
+    """bench.py places the e2e host buffers on the GPU's NUMA node from the
+    device's sysfs cpulist."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+    assert bench.parse_cpulist("") == set()
